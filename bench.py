@@ -1,0 +1,448 @@
+#!/usr/bin/env python
+"""Throughput of the absorbed-MLA decode path on B200.
+
+One step = the whole hot path over one batch of the dense decode workload (B=32
+sequences, q_len=1, 8192 cached latent rows each, 64 heads, 256-dim NoPE heads, latent
+512, bf16, seed 0): query absorption (q~ = W_UK^T q), split-L latent attention with the
+log-sum-exp combine, and the W_UV up-projection.  ``value`` is the effective HBM
+bandwidth of a step: the algorithmic bytes (every visible cache row read once, 1,024 B,
+plus both weight matrices, q, and the output) divided by the device time of a step;
+with N ranks every rank runs its own batch (weak scaling, no collective on the data
+path) and value sums the bytes over ranks divided by the slowest rank's time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
+
+``--impl reference`` times the fp64 CPU oracle (test infrastructure) on a bounded sample
+of the same workload instead; it is the reported CPU baseline.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "latent-cache attention: effective HBM GB/s & TFLOP/s vs B200 roofline, 1 GPU"
+UNIT = "GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic of one attend launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
+# ncu capture summarised in profiles/, keyed by the hash of the kernel source it was taken on.
+TRAFFIC = {}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="dense_decode")
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU-oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- workload accounting
+
+def step_bytes(wl) -> dict:
+    """Algorithmic bytes of one step: each visible cache row once (1,024 B), both weights,
+    q in, o_latent/q~ round trips excluded (intermediates), out written."""
+    H, D, R = 64, 256, 512
+    if wl.mode == "indexed":
+        rows = wl.B * wl.Q * wl.indices.shape[2]
+    elif wl.Q == 1:
+        rows = int(sum(int(L) for L in wl.seq_lens))
+    else:
+        rows = int(sum(int(L) for L in wl.seq_lens))  # all Q queries share each row's single read
+    visible_pairs = 0
+    for L in wl.seq_lens:
+        for i in range(wl.Q):
+            visible_pairs += (wl.indices.shape[2] if wl.mode == "indexed" else int(L) - wl.Q + i + 1)
+    cache = rows * R * 2
+    weights = 2 * H * D * R * 2
+    qio = 2 * wl.B * wl.Q * H * D * 2
+    flops_attend = visible_pairs * H * 4 * R
+    flops_proj = 2 * (2 * wl.B * wl.Q * H * D * R)
+    return {"cache": cache, "total": cache + weights + qio, "flops_attend": flops_attend,
+            "flops_total": flops_attend + flops_proj}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for fn in ("attend.cu", "sm100.cuh", "internal.h"):
+        with open(os.path.join(ROOT, "mla_absorbed_latent_mtp_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = []
+        for ts, line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+            except ValueError:
+                continue
+        window = [r for r in rows if t0 <= r[0] <= t1] or rows
+        if not window:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in window for k, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in window), "sm_max_mhz": max(r[2] for r in window),
+                "reasons": reasons, "samples": len(window)}
+
+
+# ----------------------------------------------------------------------------- distributed helpers
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(values, device):
+    """Element-wise max over ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized():
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def reduce_sum(values, device):
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized():
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return t.tolist()
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def aggregate(local_ms, local_bytes, device):
+    """Whole-job throughput: bytes summed over ranks / slowest rank's time."""
+    (ms,) = reduce_max([local_ms], device)
+    (total_bytes,) = reduce_sum([float(local_bytes)], device)
+    return ms, total_bytes / (ms * 1e-3) / 1e9
+
+
+# ----------------------------------------------------------------------------- CPU oracle baseline
+
+def cpu_baseline(wl, budget_s):
+    """Time the fp64 oracle (expanded form, as it stands) on a bounded sample: heads of
+    sequence 0, query 0, added until the budget is spent.  Reported in the metric's unit."""
+    import numpy as np  # noqa: F401
+    import oracle
+    t_start = time.perf_counter()
+    heads = 0
+    while heads < 64:
+        oracle.reference(wl, pairs=[(0, 0)], heads=[heads], row_source=None)
+        heads += 1
+        if time.perf_counter() - t_start > budget_s:
+            break
+    dt = time.perf_counter() - t_start
+    L = int(wl.seq_lens[0]) if wl.mode != "indexed" else wl.indices.shape[2]
+    bytes_attributed = L * 1024 * heads / 64.0
+    cores = threads_used()
+    return {"value": bytes_attributed / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"sequence 0, query 0, {heads} of 64 heads, {L} cached rows, expanded fp64 form "
+                      f"({dt:.1f} s)"}
+
+
+def threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("internal_api") in ("openblas", "mkl", "blis")]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args, wl_name):
+    """The oracle on the host cores, each step a bounded sample (one head of one sequence)."""
+    import synth
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    wl = synth.make_workload(wl_name, with_data=False)
+    import oracle
+
+    L = int(wl.seq_lens[0]) if wl.mode != "indexed" else wl.indices.shape[2]
+    rows_fn = lambda b, pos: synth.cache_rows(wl, b, pos)  # noqa: E731
+    budget_total = 150.0
+    # calibrate the rows per step so that warmup + steps fit the budget
+    rows = L
+    t = time.perf_counter()
+    sub = _truncated(wl, rows)
+    oracle.reference(sub, pairs=[(0, sub.Q - 1)], heads=[0], row_source=rows_fn)
+    one = time.perf_counter() - t
+    per_step = budget_total / max(args.steps + args.warmup, 1)
+    if one > per_step:
+        rows = max(64, int(L * per_step / one))
+        sub = _truncated(wl, rows)
+    for _ in range(args.warmup):
+        oracle.reference(sub, pairs=[(0, sub.Q - 1)], heads=[0], row_source=rows_fn)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.reference(sub, pairs=[(0, sub.Q - 1)], heads=[0], row_source=rows_fn)
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    value = rows * 1024 / 64.0 / dt / 1e9
+    sample = f"one head of sequence 0 (last query), {rows} cached rows per step, expanded fp64 form"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl_name, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads_used(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def _truncated(wl, rows):
+    """Same workload restricted to its first `rows` cache rows of sequence 0."""
+    import copy
+    sub = copy.copy(wl)
+    import numpy as np
+    lens = wl.seq_lens.copy()
+    if wl.mode != "indexed":
+        lens[0] = min(int(lens[0]), rows)
+    else:
+        sub.indices = wl.indices[:, :, :rows]
+    sub.seq_lens = lens
+    return sub
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        if world > 1:
+            import torch.distributed as dist
+            dist.init_process_group("gloo")
+            run_reference(args, args.config)
+            dist.destroy_process_group()
+        else:
+            run_reference(args, args.config)
+        return
+
+    import numpy as np
+    import torch
+
+    import mla_absorbed_latent_mtp_b200 as m
+    import synth
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    from mla_absorbed_latent_mtp_b200 import _build
+    if rank == 0:
+        _build.build()
+    barrier()
+    m.lib()
+
+    wl = synth.make_workload(args.config, seed=rank, with_data=False)
+    acc = step_bytes(wl)
+    B, Q = wl.B, wl.Q
+
+    def dev_bits(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
+
+    host_cache = torch.empty(wl.extra["cache_shape"], dtype=torch.int16, pin_memory=True)
+    synth.fill_cache(wl, host_cache.data_ptr())
+    host_q = torch.from_numpy(np.ascontiguousarray(wl.q).view(np.int16)).pin_memory()
+    cache = host_cache.to(device).view(torch.bfloat16)
+    q = host_q.to(device).view(torch.bfloat16)
+    w_uk, w_uv = dev_bits(wl.w_uk), dev_bits(wl.w_uv)
+    lens = torch.from_numpy(wl.seq_lens).to(device)
+    host_lens = torch.from_numpy(wl.seq_lens).pin_memory()
+    table = torch.from_numpy(wl.page_table).to(device) if wl.mode == "paged" else None
+    idx = torch.from_numpy(wl.indices).to(device) if wl.mode == "indexed" else None
+    ws = m.new_workspace(B, Q)
+    qt = torch.empty(B, Q, 64, 512, dtype=torch.bfloat16, device=device)
+    o = torch.empty(B, Q, 64, 512, dtype=torch.bfloat16, device=device)
+    lse = torch.empty(B, Q, 64, dtype=torch.float32, device=device)
+    out = torch.empty(B, Q, 64, 256, dtype=torch.bfloat16, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    host_out = torch.empty(out.shape, dtype=torch.int16, pin_memory=True)
+
+    def absorb():
+        m.mla_absorb_q(q, w_uk, qt)
+
+    def attend():
+        if wl.mode == "dense":
+            m.mla_attend_dense(qt, cache, lens, wl.scale, ws, o, lse, status)
+        elif wl.mode == "paged":
+            m.mla_attend_paged(qt, cache, table, lens, wl.scale, ws, o, lse, status)
+        else:
+            m.mla_attend_indexed(qt, cache, idx, lens, wl.scale, ws, o, lse, status)
+
+    def up():
+        m.mla_up_proj(o, w_uv, out)
+
+    for _ in range(args.warmup):
+        absorb(); attend(); up()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, m.status_string(int(status.item()))
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    start.record()
+    for k in range(K):
+        e = ev[k]
+        e[0].record(); absorb(); e[1].record(); attend(); e[2].record(); up(); e[3].record()
+    stop.record()
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    barrier()
+    time.sleep(0.1)
+    clocks.stop()
+    local_ms = start.elapsed_time(stop) / K
+    stage = [sum(ev[k][j].elapsed_time(ev[k][j + 1]) for k in range(K)) / K for j in range(3)]
+    ms, value = aggregate(local_ms, acc["total"], device)
+    stage = reduce_max(stage, device)
+    launches = K * 4  # absorb, attend, combine, up-projection
+
+    # end to end through the public API with host buffers: H2D inputs, D2H output per step
+    Ke = max(1, min(args.e2e_steps, K))
+    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h2d = host_cache.numel() * 2 + host_q.numel() * 2 + host_lens.numel() * 4
+    d2h = host_out.numel() * 2
+    barrier()
+    torch.cuda.synchronize()
+    e_start.record()
+    for _ in range(Ke):
+        cache.view(torch.int16).copy_(host_cache, non_blocking=True)
+        q.view(torch.int16).copy_(host_q, non_blocking=True)
+        lens.copy_(host_lens, non_blocking=True)
+        absorb(); attend(); up()
+        host_out.copy_(out.view(torch.int16), non_blocking=True)
+    e_stop.record()
+    torch.cuda.synchronize()
+    e_ms, e_value = aggregate(e_start.elapsed_time(e_stop) / Ke, acc["total"], device)
+    assert int(status.item()) == 0, m.status_string(int(status.item()))
+
+    peaks, peak_kind = load_peaks()
+    att_gbs = acc["cache"] / (stage[1] * 1e-3) / 1e9
+    src_hash = kernel_source_hash()
+    traffic = TRAFFIC.get((args.config, src_hash))
+    roofline = {"bound": "hbm", "achieved": att_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": att_gbs / peaks["hbm_gbs"], "traffic": traffic,
+                "kernel": "attend_kernel + combine_kernel (mla_attend_*)", "peak_source": peak_kind}
+    t_mem = acc["cache"] / (peaks["hbm_gbs"] * 1e9)
+    t_tc = acc["flops_attend"] / (peaks["bf16_tflops"] * 1e12)
+    if t_tc > t_mem:
+        ach = acc["flops_attend"] / (stage[1] * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": ach / peaks["bf16_tflops"], "traffic": traffic,
+                    "kernel": "attend_kernel + combine_kernel (mla_attend_*)", "peak_source": peak_kind}
+
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded SplitMix64/Box-Muller; random-init weights of the stated shapes)",
+        "config": {"workload": args.config, "B": B, "q_len": Q, "mode": wl.mode,
+                   "cache_rows": int(sum(int(x) for x in wl.seq_lens)) if wl.mode != "indexed" else None,
+                   "heads": 64, "head_dim": 256, "latent": 512, "parallelism": f"dp{world} (independent batches)",
+                   "l2": "inputs larger than L2 (cache %.0f MB per rank)" % (acc["cache"] / 1e6)},
+        "stages_ms": {"absorb_q": stage[0], "attend": stage[2 - 1], "up_proj": stage[2]},
+        "attend_tflops": acc["flops_attend"] / (stage[1] * 1e-3) / 1e12,
+        "roofline": roofline,
+        "e2e": {"value": e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e_ms, "steps": Ke},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(wall0, wall1),
+        "kernel_src": src_hash,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        wl_cpu = synth.make_workload(args.config, with_data=False)
+        wl_cpu.cache = host_cache.numpy().view(np.uint16) if wl.mode != "paged" else None
+        wl_cpu.pool = host_cache.numpy().view(np.uint16) if wl.mode == "paged" else None
+        result["cpu_baseline"] = cpu_baseline(wl_cpu, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(result))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

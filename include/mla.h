@@ -1,0 +1,146 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) absorbed Multi-head Latent Attention library.
+ *
+ * The operation is attention over a latent cache in its absorbed form, as derived
+ * on the page "Module 05 -- MLA: Compressing Per-Token History" (jared-hpc.com,
+ * GLM-5.3-Flash Architecture Mastery, Lecture-05):
+ *   section 1  every cached token keeps one shared latent c_j (width R = 512);
+ *              per head h the key/value are k = U_h^K c_j and v = U_h^V c_j,
+ *              U_h in R^{D x R} with D = 256 and H = 64 heads (NoPE);
+ *   section 3  q~_h = (U_h^K)^T q_h  (mla_absorb_q),
+ *              score_j = scale * q~_h . c_j, softmax, o_h = sum_j a_j c_j
+ *              (mla_attend_*), out_h = U_h^V o_h (mla_up_proj);
+ *              the scale is the original q.k temperature (1/sqrt(256) = 1/16);
+ *   section 4  causal masking: a query at position t sees positions j <= t.
+ * Multi-token-prediction verification (page dimsnsums.com/models/glm-5-3-flash/mtp)
+ * scores all q_len = 1 + drafts positions of a proposed run in one pass: with the
+ * q_len new latents already appended to a cache of L_b rows, query i sits at
+ * position t_i = L_b - q_len + i and sees rows 0..t_i.
+ *
+ * Conventions for every entry point
+ *  - bf16 tensors are passed as uint16_t bit patterns; all tensors are dense,
+ *    row-major (last index fastest) and 16-byte aligned.
+ *  - Every data pointer is a DEVICE pointer owned by the caller.  The library never
+ *    allocates, frees, synchronises or throws; work is enqueued on `stream`
+ *    (a cudaStream_t, NULL = legacy default stream) and runs asynchronously.
+ *  - Host-detectable errors (null pointers, bad sizes, unsupported H/D/R,
+ *    misalignment, workspace too small) return an error code and enqueue nothing.
+ *  - Device-detectable errors (page id or index out of range, a bounded wait that
+ *    expired) are written to *status (a device int32, may be NULL) only if it is still
+ *    MLA_OK, so the first error is kept; the caller zeroes it and reads it after its
+ *    own synchronisation.  Outputs are unspecified when *status != MLA_OK.
+ *  - Supported sizes in this version: H = 64, D = 256, R = 512.
+ */
+#ifndef MLA_B200_H
+#define MLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t mla_status;
+
+#define MLA_OK 0
+#define MLA_ERR_ARG 1          /* null pointer, non-positive or inconsistent size */
+#define MLA_ERR_UNSUPPORTED 2  /* H, D or R other than 64, 256, 512; misaligned pointer */
+#define MLA_ERR_CUDA 3         /* a CUDA runtime/driver call failed (launch, tensor map) */
+#define MLA_ERR_WORKSPACE 4    /* workspace pointer null or ws_bytes too small */
+#define MLA_ERR_INDEX 5        /* device: page id / cache index / length out of range */
+#define MLA_ERR_TIMEOUT 6      /* device: a bounded pipeline wait expired */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *mla_status_string(mla_status s);
+
+/*
+ * Query absorption, Module 05 section 3:  q_tilde[n,h,:] = U_h^K^T q[n,h,:].
+ *   q       [n, H, D] bf16     query heads (n = batch * q_len rows)
+ *   w_uk    [H, D, R] bf16     U^K per head, k = U_h^K c  (row d, column r)
+ *   q_tilde [n, H, R] bf16     output, fp32 accumulation, rounded to nearest even
+ * n >= 1.  Errors: MLA_ERR_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_CUDA.
+ */
+mla_status mla_absorb_q(const uint16_t *q, const uint16_t *w_uk, uint16_t *q_tilde,
+                        int n, int H, int D, int R, void *stream);
+
+/*
+ * Latent attention over a contiguous cache, Module 05 sections 3-4 (+ MTP window).
+ *   q_tilde  [B, Q, H, R] bf16   absorbed queries (output of mla_absorb_q)
+ *   cache    [B, Lmax, R] bf16   latent rows c_j of each sequence
+ *   seq_lens [B] int32 or NULL   rows L_b of sequence b, INCLUDING the Q newly appended
+ *                                query rows; NULL means every sequence has Lmax rows.
+ *                                0 <= L_b <= Lmax (else MLA_ERR_INDEX on *status).
+ *   scale                         softmax scale applied to q~.c (1/16 for these heads)
+ *   workspace, ws_bytes           caller scratch, >= mla_attend_workspace_bytes(B, Q, H, R)
+ *   o_latent [B, Q, H, R] bf16   o = sum_j a_j c_j (normalised), the input of mla_up_proj
+ *   lse      [B, Q, H] fp32      natural-log sum-exp of the scaled scores, or NULL
+ * Query i of sequence b sees rows 0 .. L_b - Q + i; an empty window gives o = 0 and
+ * lse = -inf.  Rows beyond L_b may hold any bits (they are never used).
+ */
+mla_status mla_attend_dense(const uint16_t *q_tilde, const uint16_t *cache, const int32_t *seq_lens,
+                            int B, int Q, int H, int R, int Lmax, float scale,
+                            void *workspace, size_t ws_bytes, uint16_t *o_latent, float *lse,
+                            int32_t *status, void *stream);
+
+/*
+ * Same as mla_attend_dense over a paged cache: logical row j of sequence b is
+ *   pool[page_table[b * max_pages + j / page_size]][j % page_size][:].
+ *   pool       [num_pages, page_size, R] bf16
+ *   page_table [B, max_pages] int32   entries for pages past the end are ignored
+ *   seq_lens   [B] int32 (required)   0 <= L_b <= max_pages * page_size
+ * page_size must be 64.  A used entry outside [0, num_pages) sets MLA_ERR_INDEX.
+ * The result is bit-identical to mla_attend_dense on the same logical rows.
+ */
+mla_status mla_attend_paged(const uint16_t *q_tilde, const uint16_t *pool, const int32_t *page_table,
+                            const int32_t *seq_lens, int B, int Q, int H, int R, int page_size,
+                            int max_pages, int num_pages, float scale, void *workspace, size_t ws_bytes,
+                            uint16_t *o_latent, float *lse, int32_t *status, void *stream);
+
+/*
+ * Attention of each query over a given list of cache positions (a sparse selection
+ * such as the DSA indexer's): query i of sequence b attends exactly to the rows
+ * cache[b, indices[b, i, k]] for k < K.
+ *   indices  [B, Q, K] int32   positions, each in [0, L_b - Q + i] (causally visible);
+ *                              order does not matter, a repeated entry counts twice.
+ *   seq_lens [B] int32 or NULL  as for mla_attend_dense (used to validate indices)
+ * An out-of-range entry sets MLA_ERR_INDEX.  K >= 1.
+ */
+mla_status mla_attend_indexed(const uint16_t *q_tilde, const uint16_t *cache, const int32_t *indices,
+                              const int32_t *seq_lens, int B, int Q, int H, int R, int Lmax, int K,
+                              float scale, void *workspace, size_t ws_bytes, uint16_t *o_latent,
+                              float *lse, int32_t *status, void *stream);
+
+/*
+ * Value up-projection, Module 05 section 3:  out[n,h,:] = U_h^V o_latent[n,h,:].
+ *   o_latent [n, H, R] bf16, w_uv [H, D, R] bf16 (v = U_h^V c), out [n, H, D] bf16.
+ */
+mla_status mla_up_proj(const uint16_t *o_latent, const uint16_t *w_uv, uint16_t *out,
+                       int n, int H, int D, int R, void *stream);
+
+/*
+ * Bytes of workspace the mla_attend_* calls need for B sequences of Q queries on the
+ * current device (split-L partial results and their max/sum terms).  0 on bad sizes.
+ */
+size_t mla_attend_workspace_bytes(int B, int Q, int H, int R);
+
+/*
+ * Test aid: copy the latent rows the attend kernels would address, with the same
+ * address computation, so that page-table and index handling can be compared bit
+ * for bit.  For request r = (req[3r], req[3r+1], req[3r+2]) = (b, i, k):
+ *   mode 0 (dense):   out[r] = cache[b, k]
+ *   mode 1 (paged):   out[r] = pool[page_table[b, k / 64], k % 64]
+ *   mode 2 (indexed): out[r] = cache[b, indices[b, i, k]]
+ * `src` is the cache (modes 0, 2) or the pool (mode 1); sizes as in the attend calls
+ * (Lmax is unused in mode 1, num_pages unused in modes 0 and 2).  A request whose
+ * address is out of range writes a zero row and sets MLA_ERR_INDEX on *status.
+ */
+mla_status mla_debug_gather(int mode, const uint16_t *src, const int32_t *page_table, const int32_t *indices,
+                            int B, int Q, int R, int Lmax, int max_pages, int num_pages, int K,
+                            const int32_t *req, int n_req, uint16_t *out, int32_t *status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H */

@@ -1,0 +1,200 @@
+"""Python binding of the B200 absorbed-MLA latent attention library (include/mla.h).
+
+Argument marshalling only: every step runs in the CUDA kernels of libmla_b200.so.
+Tensors are torch CUDA tensors (bf16 as torch.bfloat16, int32 as torch.int32); the
+functions pass their device pointers and the current CUDA stream to the C ABI and
+raise MLAError on a non-zero status.  There is no CPU fallback: if the library is
+not built, importing the binding's functions raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmla_b200.so")
+
+MLA_OK, MLA_ERR_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_CUDA, MLA_ERR_WORKSPACE, MLA_ERR_INDEX, MLA_ERR_TIMEOUT = range(7)
+MODE_DENSE, MODE_PAGED, MODE_INDEXED = 0, 1, 2
+H, D, R, PAGE = 64, 256, 512, 64
+SCALE = 1.0 / 16.0
+
+EXPORTS = ("mla_status_string", "mla_absorb_q", "mla_attend_dense", "mla_attend_paged", "mla_attend_indexed",
+           "mla_up_proj", "mla_attend_workspace_bytes", "mla_debug_gather")
+
+
+class MLAError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} failed: {status_string(code)} ({code})")
+        self.code = code
+
+
+_lib = None
+
+
+def lib():
+    """The loaded shared library (ctypes), with argument types declared."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run: python -c 'import __graft_entry__ as g; g.build()'")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    L.mla_status_string.argtypes = [ctypes.c_int32]
+    L.mla_status_string.restype = ctypes.c_char_p
+    L.mla_absorb_q.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
+    L.mla_up_proj.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
+    L.mla_attend_dense.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, sz, vp, vp, vp, vp]
+    L.mla_attend_paged.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, vp, sz, vp, vp, vp, vp]
+    L.mla_attend_indexed.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, sz, vp, vp, vp, vp]
+    L.mla_attend_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    L.mla_attend_workspace_bytes.restype = sz
+    L.mla_debug_gather.argtypes = [i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp]
+    for name in ("mla_absorb_q", "mla_up_proj", "mla_attend_dense", "mla_attend_paged", "mla_attend_indexed",
+                 "mla_debug_gather"):
+        getattr(L, name).restype = ctypes.c_int32
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return lib().mla_status_string(code).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, code):
+    if code != MLA_OK:
+        raise MLAError(fn, code)
+
+
+def _check_cuda(*tensors):
+    for t in tensors:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors")
+
+
+# ----------------------------------------------------------------------------- entry points
+
+def mla_attend_workspace_bytes(B: int, Q: int, heads: int = H, latent: int = R) -> int:
+    return int(lib().mla_attend_workspace_bytes(B, Q, heads, latent))
+
+
+def new_workspace(B: int, Q: int):
+    """Allocate (with torch) the workspace the attend calls need."""
+    import torch
+    n = mla_attend_workspace_bytes(B, Q)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+
+
+def mla_absorb_q(q, w_uk, q_tilde=None, stream=None):
+    """q [n, H, D] or [B, Q, H, D] bf16, w_uk [H, D, R] bf16 -> q_tilde [..., H, R] bf16."""
+    import torch
+    _check_cuda(q, w_uk, q_tilde)
+    n = q.numel() // (H * D)
+    if q_tilde is None:
+        q_tilde = torch.empty(*q.shape[:-1], R, dtype=torch.bfloat16, device=q.device)
+    _check("mla_absorb_q", lib().mla_absorb_q(_ptr(q), _ptr(w_uk), _ptr(q_tilde), n, H, D, R, _stream(stream)))
+    return q_tilde
+
+
+def mla_up_proj(o_latent, w_uv, out=None, stream=None):
+    """o_latent [..., H, R] bf16, w_uv [H, D, R] bf16 -> out [..., H, D] bf16."""
+    import torch
+    _check_cuda(o_latent, w_uv, out)
+    n = o_latent.numel() // (H * R)
+    if out is None:
+        out = torch.empty(*o_latent.shape[:-1], D, dtype=torch.bfloat16, device=o_latent.device)
+    _check("mla_up_proj", lib().mla_up_proj(_ptr(o_latent), _ptr(w_uv), _ptr(out), n, H, D, R, _stream(stream)))
+    return out
+
+
+def _attend_outputs(q_tilde, o_latent, lse, want_lse):
+    import torch
+    B, Q = q_tilde.shape[0], q_tilde.shape[1]
+    if o_latent is None:
+        o_latent = torch.empty(B, Q, H, R, dtype=torch.bfloat16, device=q_tilde.device)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Q, H, dtype=torch.float32, device=q_tilde.device)
+    return o_latent, lse
+
+
+def mla_attend_dense(q_tilde, cache, seq_lens=None, scale=SCALE, workspace=None, o_latent=None, lse=None,
+                     status=None, want_lse=True, stream=None):
+    """q_tilde [B, Q, H, R], cache [B, Lmax, R] (bf16), seq_lens [B] int32 or None."""
+    _check_cuda(q_tilde, cache, seq_lens, workspace, o_latent, lse, status)
+    B, Q = q_tilde.shape[0], q_tilde.shape[1]
+    Lmax = cache.shape[1]
+    workspace = new_workspace(B, Q) if workspace is None else workspace
+    o_latent, lse = _attend_outputs(q_tilde, o_latent, lse, want_lse)
+    _check("mla_attend_dense", lib().mla_attend_dense(
+        _ptr(q_tilde), _ptr(cache), _ptr(seq_lens), B, Q, H, R, Lmax, scale, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(o_latent), _ptr(lse), _ptr(status), _stream(stream)))
+    return o_latent, lse
+
+
+def mla_attend_paged(q_tilde, pool, page_table, seq_lens, scale=SCALE, workspace=None, o_latent=None, lse=None,
+                     status=None, want_lse=True, stream=None):
+    """pool [P, 64, R] bf16, page_table [B, max_pages] int32, seq_lens [B] int32."""
+    _check_cuda(q_tilde, pool, page_table, seq_lens, workspace, o_latent, lse, status)
+    B, Q = q_tilde.shape[0], q_tilde.shape[1]
+    workspace = new_workspace(B, Q) if workspace is None else workspace
+    o_latent, lse = _attend_outputs(q_tilde, o_latent, lse, want_lse)
+    _check("mla_attend_paged", lib().mla_attend_paged(
+        _ptr(q_tilde), _ptr(pool), _ptr(page_table), _ptr(seq_lens), B, Q, H, R, pool.shape[1],
+        page_table.shape[1], pool.shape[0], scale, _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(o_latent), _ptr(lse), _ptr(status), _stream(stream)))
+    return o_latent, lse
+
+
+def mla_attend_indexed(q_tilde, cache, indices, seq_lens=None, scale=SCALE, workspace=None, o_latent=None, lse=None,
+                       status=None, want_lse=True, stream=None):
+    """cache [B, Lmax, R] bf16, indices [B, Q, K] int32."""
+    _check_cuda(q_tilde, cache, indices, seq_lens, workspace, o_latent, lse, status)
+    B, Q = q_tilde.shape[0], q_tilde.shape[1]
+    workspace = new_workspace(B, Q) if workspace is None else workspace
+    o_latent, lse = _attend_outputs(q_tilde, o_latent, lse, want_lse)
+    _check("mla_attend_indexed", lib().mla_attend_indexed(
+        _ptr(q_tilde), _ptr(cache), _ptr(indices), _ptr(seq_lens), B, Q, H, R, cache.shape[1], indices.shape[2],
+        scale, _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(o_latent), _ptr(lse),
+        _ptr(status), _stream(stream)))
+    return o_latent, lse
+
+
+def mla_debug_gather(mode, src, req, page_table=None, indices=None, B=None, Q=1, Lmax=0, status=None, stream=None):
+    """Rows the attend kernels would address for requests req [n, 3] int32 (b, i, k)."""
+    import torch
+    _check_cuda(src, req, page_table, indices, status)
+    n = req.shape[0]
+    out = torch.empty(n, R, dtype=torch.bfloat16, device=src.device)
+    max_pages = page_table.shape[1] if page_table is not None else 0
+    num_pages = src.shape[0] if mode == MODE_PAGED else 0
+    K = indices.shape[2] if indices is not None else 0
+    _check("mla_debug_gather", lib().mla_debug_gather(
+        mode, _ptr(src), _ptr(page_table), _ptr(indices), B, Q, R, Lmax, max_pages, num_pages, K, _ptr(req), n,
+        _ptr(out), _ptr(status), _stream(stream)))
+    return out
+
+
+def mla_decode(q, w_uk, w_uv, cache, seq_lens=None, *, mode=MODE_DENSE, page_table=None, indices=None,
+               scale=SCALE, workspace=None, status=None, stream=None):
+    """The whole path: absorb -> attend (dense / paged / indexed) -> up-project.
+
+    q [B, Q, H, D] bf16 -> out [B, Q, H, D] bf16 (and lse [B, Q, H])."""
+    qt = mla_absorb_q(q, w_uk, stream=stream)
+    if mode == MODE_DENSE:
+        o, lse = mla_attend_dense(qt, cache, seq_lens, scale, workspace, status=status, stream=stream)
+    elif mode == MODE_PAGED:
+        o, lse = mla_attend_paged(qt, cache, page_table, seq_lens, scale, workspace, status=status, stream=stream)
+    else:
+        o, lse = mla_attend_indexed(qt, cache, indices, seq_lens, scale, workspace, status=status, stream=stream)
+    return mla_up_proj(o, w_uv, stream=stream), lse

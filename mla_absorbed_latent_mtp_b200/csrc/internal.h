@@ -1,0 +1,57 @@
+// internal.h -- host-side declarations shared by the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mla {
+
+// Address modes of the attend kernel.
+enum AttendMode : int { kModeDense = 0, kModePaged = 1, kModeIndexed = 2 };
+
+// Fixed problem geometry of this version (Module 05 section 1).
+constexpr int kHeads = 64;
+constexpr int kHeadDim = 256;
+constexpr int kLatent = 512;
+constexpr int kPageTokens = 64;
+
+// Everything the attend and combine kernels need besides the two tensor maps.
+struct AttendParams {
+  const int32_t *seq_lens;    // [B] or null (dense/indexed: every sequence has Lmax rows)
+  const int32_t *page_table;  // paged: [B, max_pages]
+  const int32_t *indices;     // indexed: [B, Q, K]
+  const uint16_t *cache;      // indexed: raw pointer of the [B, Lmax, R] cache
+  int B, Q, Lmax, max_pages, num_pages, K;
+  int groups;                 // G: CTA groups that split the tile list
+  int group_size;             // CTAs per group: Q (dense/paged, one per query) or 1 (indexed)
+  float scale_log2;           // softmax scale * log2(e)
+  float *part_o;              // [slots, H, R] unnormalised partial outputs
+  float *part_m;              // [slots, H] running max (log2 units)
+  float *part_l;              // [slots, H] running sum
+  uint16_t *o_latent;         // [B, Q, H, R] result
+  float *lse;                 // [B, Q, H] or null
+  int32_t *status;
+};
+
+// Partial-result slots needed for B sequences of Q queries with `sms` SMs.
+size_t attend_slots(int B, int Q, int sms);
+size_t attend_workspace_bytes_for(int B, int Q, int sms);
+
+cudaError_t launch_attend(int mode, const CUtensorMap &tm_cache, const CUtensorMap &tm_qt,
+                          const AttendParams &p, cudaStream_t stream);
+cudaError_t launch_debug_gather(int mode, const uint16_t *src, const int32_t *page_table,
+                                const int32_t *indices, int B, int Q, int R, int Lmax, int max_pages,
+                                int num_pages, int K, const int32_t *req, int n_req, uint16_t *out,
+                                int32_t *status, cudaStream_t stream);
+
+// Per-head projection GEMM: out[n, h, m] = sum_k A_h[m, k] * X[n, h, k].
+// absorb (a_mn_major = true):  A_h[m=r, k=d] = W_UK[h][d][r]  (M = R, K = D)
+// up-proj (a_mn_major = false): A_h[m=d, k=r] = W_UV[h][d][r] (M = D, K = R)
+cudaError_t launch_proj(bool a_mn_major, const CUtensorMap &tm_w, const CUtensorMap &tm_x, int n, int H,
+                        int M_total, int K_total, int n_tile, uint16_t *out, cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace mla

@@ -1,0 +1,172 @@
+// proj.cu -- the two per-head projections around latent attention (Module 05, section 3):
+//   absorb:  q~[n, h, r]  = sum_d W_UK[h][d][r] * q[n, h, d]      (q~_h = U_h^K^T q_h)
+//   up-proj: out[n, h, d] = sum_r W_UV[h][d][r] * o[n, h, r]      (out_h = U_h^V o_h)
+// Both are weight-streaming GEMMs with few token rows, so the weights go on the MMA M
+// side (128 rows per CTA) and the tokens on N:
+//   D[m, n] = A_h[m, k] * X[n, h, k]^T,   A_h = W_UK[h]^T (MN-major) or W_UV[h] (K-major).
+// One CTA per (head, 128-row weight block, token tile): warp 0 streams 64-wide K chunks
+// through a 4-stage TMA ring, warp 1 issues tcgen05 MMAs into TMEM, warps 2-5 convert the
+// fp32 accumulator to bf16 and store it.
+#include <algorithm>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace mla {
+namespace proj {
+
+constexpr int kThreads = 192;
+constexpr int kStages = 4;
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kMaxNT = 128;
+constexpr int kABytes = kBM * kBK * 2;      // 16 KB per stage
+constexpr int kBBytesMax = kMaxNT * kBK * 2; // 16 KB per stage
+constexpr int kOffA = 0;
+constexpr int kOffB = kOffA + kStages * kABytes;
+constexpr int kOffBar = kOffB + kStages * kBBytesMax;
+constexpr int kOffMisc = kOffBar + (2 * kStages + 1) * 8;
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+constexpr uint32_t kTmemCols = 128;
+
+struct Params {
+  int n, H, M_total, K_total, n_tile;
+  uint16_t *out;
+};
+
+template <bool kAMajorMN>
+__global__ void __launch_bounds__(kThreads, 1)
+    proj_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(base + kOffBar);
+  uint64_t *empty = full + kStages;
+  uint64_t *done = empty + kStages;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kOffMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(base + kOffMisc + 4);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int h = blockIdx.x, mb = blockIdx.y, nt = blockIdx.z;
+  const int NT = p.n_tile;
+  const int nk = p.K_total / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&tm_w);
+      prefetch_tensormap(&tm_x);
+      for (int kc = 0; kc < nk; ++kc) {
+        const int s = kc % kStages, use = kc / kStages;
+        if (!mbar_wait(&empty[s], (use & 1) ^ 1, abort_flag, nullptr)) break;
+        mbar_arrive_expect_tx(&full[s], kABytes + NT * kBK * 2);
+        uint8_t *a_dst = base + kOffA + s * kABytes;
+        if (kAMajorMN) {
+          // W_UK[h][d][r]: box {64 r, 64 d}; two boxes cover the 128 r of this block
+          tma_load_3d(a_dst, &tm_w, &full[s], mb * kBM, kc * kBK, h);
+          tma_load_3d(a_dst + kABytes / 2, &tm_w, &full[s], mb * kBM + 64, kc * kBK, h);
+        } else {
+          // W_UV[h][d][r]: box {64 r, 128 d}
+          tma_load_3d(a_dst, &tm_w, &full[s], kc * kBK, mb * kBM, h);
+        }
+        tma_load_3d(base + kOffB + s * kBBytesMax, &tm_x, &full[s], kc * kBK, h, nt * NT);
+      }
+    }
+  } else if (warp == 1) {
+    const uint32_t idesc = idesc_bf16_f32(kBM, NT, kAMajorMN, false);
+    bool ok = true;
+    for (int kc = 0; kc < nk && ok; ++kc) {
+      const int s = kc % kStages, use = kc / kStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(&full[s], use & 1, abort_flag, nullptr));
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t a_base = smem_u32(base + kOffA + s * kABytes);
+        const uint32_t b_base = smem_u32(base + kOffB + s * kBBytesMax);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          // MN-major A: 64-wide r atoms 8 KB apart (LBO), 8-row d groups 1 KB apart (SBO);
+          // K-major A/B: 128-byte rows, 8-row groups 1 KB apart, K step = 32 bytes.
+          const uint64_t a = kAMajorMN ? sw128_desc(a_base + kk * 2048, kABytes / 2, 1024)
+                                       : sw128_desc(a_base + kk * 32, 16, 1024);
+          const uint64_t b = sw128_desc(b_base + kk * 32, 16, 1024);
+          umma_bf16(tmem, a, b, idesc, (kc | kk) != 0);
+        }
+        umma_commit(&empty[s]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) umma_commit(done);
+    __syncwarp();
+  } else {
+    const bool ok = mbar_wait(done, 0, abort_flag, nullptr);
+    tc_fence_after();
+    const int wq = warp & 3;
+    const int m = mb * kBM + wq * 32 + lane;
+    for (int n0 = 0; n0 < NT; n0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + n0, r);
+      tmem_ld_wait();
+      if (ok) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int n = nt * NT + n0 + j;
+          if (n < p.n) {
+            const uint32_t v = pack_bf16x2(__uint_as_float(r[j]), 0.f);
+            p.out[((long long)n * p.H + h) * p.M_total + m] = (uint16_t)(v & 0xFFFFu);
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace proj
+
+template <bool kAMajorMN>
+static cudaError_t launch_proj_t(const CUtensorMap &tm_w, const CUtensorMap &tm_x, const proj::Params &p,
+                                 cudaStream_t stream) {
+  static int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(proj::proj_kernel<kAMajorMN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         proj::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  dim3 grid(p.H, p.M_total / proj::kBM, (p.n + p.n_tile - 1) / p.n_tile);
+  proj::proj_kernel<kAMajorMN><<<grid, proj::kThreads, proj::kSmemBytes, stream>>>(tm_w, tm_x, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_proj(bool a_mn_major, const CUtensorMap &tm_w, const CUtensorMap &tm_x, int n, int H,
+                        int M_total, int K_total, int n_tile, uint16_t *out, cudaStream_t stream) {
+  proj::Params p{n, H, M_total, K_total, n_tile, out};
+  return a_mn_major ? launch_proj_t<true>(tm_w, tm_x, p, stream) : launch_proj_t<false>(tm_w, tm_x, p, stream);
+}
+
+}  // namespace mla

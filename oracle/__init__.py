@@ -182,10 +182,9 @@ def reference(wl, pairs=None, heads=None, form: str = "expanded", row_source=Non
             union = np.unique(np.concatenate([vis[i] for i in qs])) if qs else np.zeros(0, np.int64)
         else:
             union = vis[max(qs, key=lambda i: len(vis[i]))]
-        c_all = widen(_rows(wl, b, union)) if len(union) else np.zeros((0, u_k_all.shape[2]))
+        c_all = widen(_rows(wl, b, union, row_source)) if len(union) else np.zeros((0, u_k_all.shape[2]))
         pos_to_row = {int(p): r for r, p in enumerate(union)}
         for i in qs:
-            sel = np.array([pos_to_row[int(p)] for p in vis[i]], dtype=np.int64)
             result[(b, i)] = {"out": np.zeros((len(heads), u_v_all.shape[1])), "lse": np.zeros(len(heads))}
             if return_latent:
                 result[(b, i)]["o_latent"] = np.zeros((len(heads), u_k_all.shape[2]))

@@ -1,0 +1,108 @@
+"""The C-ABI library loads on a host without a GPU, exports every symbol the header
+declares, and rejects bad host-side arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mla_absorbed_latent_mtp_b200 as m
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "mla.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import __graft_entry__
+    __graft_entry__.build()
+    return m.lib()
+
+
+def test_exports_match_header(lib):
+    declared = _declared()
+    assert set(declared) == set(m.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name)
+
+
+def test_status_strings(lib):
+    assert m.status_string(0) == "MLA_OK"
+    assert m.status_string(5) == "MLA_ERR_INDEX"
+    assert m.status_string(6) == "MLA_ERR_TIMEOUT"
+    assert m.status_string(99) == "MLA_ERR_UNKNOWN"
+
+
+def test_workspace_query_rejects_bad_sizes(lib):
+    assert lib.mla_attend_workspace_bytes(0, 1, 64, 512) == 0
+    assert lib.mla_attend_workspace_bytes(1, 0, 64, 512) == 0
+    assert lib.mla_attend_workspace_bytes(1, 1, 32, 512) == 0
+    assert lib.mla_attend_workspace_bytes(1, 1, 64, 576) == 0
+
+
+P = ctypes.c_void_p
+GOOD = P(1 << 20)  # aligned dummy address; never dereferenced on these paths
+
+
+def test_attend_rejects_host_errors(lib):
+    f = lib.mla_attend_dense
+    args = dict(qt=GOOD, c=GOOD, lens=None, B=1, Q=1, H=64, R=512, L=8, s=0.0625, ws=GOOD, wsb=1 << 30, o=GOOD)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return f(a["qt"], a["c"], a["lens"], a["B"], a["Q"], a["H"], a["R"], a["L"], a["s"], a["ws"], a["wsb"], a["o"],
+                 None, None, None)
+
+    assert call(qt=None) == m.MLA_ERR_ARG
+    assert call(o=None) == m.MLA_ERR_ARG
+    assert call(B=0) == m.MLA_ERR_ARG
+    assert call(Q=0) == m.MLA_ERR_ARG
+    assert call(H=32) == m.MLA_ERR_UNSUPPORTED
+    assert call(R=576) == m.MLA_ERR_UNSUPPORTED
+    assert call(c=P((1 << 20) + 2)) == m.MLA_ERR_UNSUPPORTED
+    assert call(L=0) == m.MLA_ERR_ARG
+    assert call(s=float("nan")) == m.MLA_ERR_ARG
+
+
+def test_paged_and_indexed_reject_host_errors(lib):
+    g = lib.mla_attend_paged
+    assert g(GOOD, GOOD, None, GOOD, 1, 1, 64, 512, 64, 4, 4, 0.0625, GOOD, 1 << 30, GOOD, None, None, None) == \
+        m.MLA_ERR_ARG
+    assert g(GOOD, GOOD, GOOD, GOOD, 1, 1, 64, 512, 32, 4, 4, 0.0625, GOOD, 1 << 30, GOOD, None, None, None) == \
+        m.MLA_ERR_UNSUPPORTED
+    h = lib.mla_attend_indexed
+    assert h(GOOD, GOOD, None, None, 1, 1, 64, 512, 8, 4, 0.0625, GOOD, 1 << 30, GOOD, None, None, None) == \
+        m.MLA_ERR_ARG
+    assert h(GOOD, GOOD, GOOD, None, 1, 1, 64, 512, 8, 0, 0.0625, GOOD, 1 << 30, GOOD, None, None, None) == \
+        m.MLA_ERR_ARG
+
+
+def test_projections_reject_host_errors(lib):
+    for f in (lib.mla_absorb_q, lib.mla_up_proj):
+        assert f(None, GOOD, GOOD, 1, 64, 256, 512, None) == m.MLA_ERR_ARG
+        assert f(GOOD, GOOD, GOOD, 0, 64, 256, 512, None) == m.MLA_ERR_ARG
+        assert f(GOOD, GOOD, GOOD, 1, 64, 128, 512, None) == m.MLA_ERR_UNSUPPORTED
+        assert f(GOOD, P((1 << 20) + 8), GOOD, 1, 64, 256, 512, None) == m.MLA_ERR_UNSUPPORTED
+
+
+def test_debug_gather_rejects_host_errors(lib):
+    f = lib.mla_debug_gather
+    assert f(3, GOOD, None, None, 1, 1, 512, 8, 0, 0, 0, GOOD, 1, GOOD, None, None) == m.MLA_ERR_ARG
+    assert f(1, GOOD, None, None, 1, 1, 512, 8, 0, 0, 0, GOOD, 1, GOOD, None, None) == m.MLA_ERR_ARG
+    assert f(0, GOOD, None, None, 1, 1, 512, 8, 0, 0, 0, GOOD, 0, GOOD, None, None) == m.MLA_OK
+
+
+def test_product_path_does_not_touch_oracle():
+    """The binding and kernels never import the oracle (test infrastructure only)."""
+    pkg = os.path.join(ROOT, "mla_absorbed_latent_mtp_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert "import oracle" not in text and "from oracle" not in text, fn
