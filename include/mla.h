@@ -54,6 +54,10 @@ typedef int32_t mla_status;
 /* Human-readable name of a status code (static string, never NULL). */
 const char *mla_status_string(mla_status s);
 
+/* Message of the last CUDA runtime error seen by an entry point on the calling thread
+ * (the reason behind an MLA_ERR_CUDA return), or "no error".  Static string. */
+const char *mla_last_error_string(void);
+
 /*
  * Query absorption, Module 05 section 3:  q_tilde[n,h,:] = U_h^K^T q[n,h,:].
  *   q       [n, H, D] bf16     query heads (n = batch * q_len rows)

@@ -19,13 +19,14 @@ MODE_DENSE, MODE_PAGED, MODE_INDEXED = 0, 1, 2
 H, D, R, PAGE = 64, 256, 512, 64
 SCALE = 1.0 / 16.0
 
-EXPORTS = ("mla_status_string", "mla_absorb_q", "mla_attend_dense", "mla_attend_paged", "mla_attend_indexed",
+EXPORTS = ("mla_status_string", "mla_last_error_string", "mla_absorb_q", "mla_attend_dense", "mla_attend_paged", "mla_attend_indexed",
            "mla_up_proj", "mla_attend_workspace_bytes", "mla_debug_gather")
 
 
 class MLAError(RuntimeError):
     def __init__(self, fn, code):
-        super().__init__(f"{fn} failed: {status_string(code)} ({code})")
+        detail = f": {lib().mla_last_error_string().decode()}" if code == MLA_ERR_CUDA else ""
+        super().__init__(f"{fn} failed: {status_string(code)} ({code}){detail}")
         self.code = code
 
 
@@ -43,6 +44,8 @@ def lib():
     vp, i32, sz, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
     L.mla_status_string.argtypes = [ctypes.c_int32]
     L.mla_status_string.restype = ctypes.c_char_p
+    L.mla_last_error_string.argtypes = []
+    L.mla_last_error_string.restype = ctypes.c_char_p
     L.mla_absorb_q.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
     L.mla_up_proj.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
     L.mla_attend_dense.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, sz, vp, vp, vp, vp]

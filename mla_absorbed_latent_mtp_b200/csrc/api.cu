@@ -60,6 +60,14 @@ int sm_count_for(int dev) {
 
 }  // namespace
 
+static thread_local cudaError_t g_last_error = cudaSuccess;
+
+static mla_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MLA_OK;
+  g_last_error = e;
+  return MLA_ERR_CUDA;
+}
+
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -86,7 +94,7 @@ static mla_status attend_common(int mode, const uint16_t *q_tilde, const uint16_
   }
   if (mode == kModeIndexed && (indices == nullptr || K < 1)) return MLA_ERR_ARG;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_status(e);
   const int sms = sm_count_for(dev);
   const size_t need = attend_workspace_bytes_for(B, Q, sms);
   if (workspace == nullptr || ws_bytes < need || !aligned16(workspace)) return MLA_ERR_WORKSPACE;
@@ -97,13 +105,13 @@ static mla_status attend_common(int mode, const uint16_t *q_tilde, const uint16_
     const uint64_t dims[2] = {(uint64_t)R, rows};
     const uint64_t strides[1] = {(uint64_t)R * 2};
     const uint32_t box[2] = {64, 64};
-    if (!make_map(&tm_cache, cache, 2, dims, strides, box)) return MLA_ERR_CUDA;
+    if (!make_map(&tm_cache, cache, 2, dims, strides, box)) return cuda_status(cudaErrorInvalidValue);
   }
   {
     const uint64_t dims[2] = {(uint64_t)R, (uint64_t)B * Q * H};
     const uint64_t strides[1] = {(uint64_t)R * 2};
     const uint32_t box[2] = {64, 64};
-    if (!make_map(&tm_qt, q_tilde, 2, dims, strides, box)) return MLA_ERR_CUDA;
+    if (!make_map(&tm_qt, q_tilde, 2, dims, strides, box)) return cuda_status(cudaErrorInvalidValue);
   }
   AttendParams p;
   p.seq_lens = seq_lens;
@@ -131,9 +139,7 @@ static mla_status attend_common(int mode, const uint16_t *q_tilde, const uint16_
   p.o_latent = o_latent;
   p.lse = lse;
   p.status = status;
-  return launch_attend(mode, tm_cache, tm_qt, p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? MLA_OK
-             : MLA_ERR_CUDA;
+  return cuda_status(launch_attend(mode, tm_cache, tm_qt, p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 static mla_status proj_common(bool absorb, const uint16_t *x, const uint16_t *w, uint16_t *out, int n, int H, int D,
@@ -153,24 +159,24 @@ static mla_status proj_common(bool absorb, const uint16_t *x, const uint16_t *w,
     const uint64_t strides[2] = {(uint64_t)R * 2, (uint64_t)D * R * 2};
     const uint32_t box_mn[3] = {64, 64, 1};
     const uint32_t box_k[3] = {64, 128, 1};
-    if (!make_map(&tm_w, w, 3, dims, strides, absorb ? box_mn : box_k)) return MLA_ERR_CUDA;
+    if (!make_map(&tm_w, w, 3, dims, strides, absorb ? box_mn : box_k)) return cuda_status(cudaErrorInvalidValue);
   }
   {
     // X[n][h][k]: dims {K, H, n}
     const uint64_t dims[3] = {(uint64_t)K_total, (uint64_t)H, (uint64_t)n};
     const uint64_t strides[2] = {(uint64_t)K_total * 2, (uint64_t)H * K_total * 2};
     const uint32_t box[3] = {64, 1, (uint32_t)n_tile};
-    if (!make_map(&tm_x, x, 3, dims, strides, box)) return MLA_ERR_CUDA;
+    if (!make_map(&tm_x, x, 3, dims, strides, box)) return cuda_status(cudaErrorInvalidValue);
   }
-  return launch_proj(absorb, tm_w, tm_x, n, H, M_total, K_total, n_tile, out,
-                     reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? MLA_OK
-             : MLA_ERR_CUDA;
+  return cuda_status(launch_proj(absorb, tm_w, tm_x, n, H, M_total, K_total, n_tile, out,
+                                 reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // namespace mla
 
 extern "C" {
+
+const char *mla_last_error_string(void) { return cudaGetErrorString(mla::g_last_error); }
 
 const char *mla_status_string(mla_status s) {
   switch (s) {
@@ -240,10 +246,8 @@ mla_status mla_debug_gather(int mode, const uint16_t *src, const int32_t *page_t
   if (mode == mla::kModeIndexed && (indices == nullptr || K < 1 || Q < 1)) return MLA_ERR_ARG;
   if (mode != mla::kModePaged && Lmax < 1) return MLA_ERR_ARG;
   if (n_req == 0) return MLA_OK;
-  return mla::launch_debug_gather(mode, src, page_table, indices, B, Q, R, Lmax, max_pages, num_pages, K, req, n_req,
-                                  out, status, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? MLA_OK
-             : MLA_ERR_CUDA;
+  return mla::cuda_status(mla::launch_debug_gather(mode, src, page_table, indices, B, Q, R, Lmax, max_pages, num_pages,
+                                                  K, req, n_req, out, status, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

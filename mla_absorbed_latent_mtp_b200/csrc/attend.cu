@@ -6,19 +6,20 @@
 // tiles of all sequences form one list that G CTA groups split into equal contiguous
 // ranges (a range may cross sequence boundaries; each piece is a "segment").  A group
 // holds one CTA per query of a verify window (Q CTAs for dense/paged caches, all reading
-// the same tiles at the same time, so the second to last read hits L2), or one CTA per
+// the same tiles at the same time, so all but the first read hit L2), or one CTA per
 // (sequence, query) list for the indexed mode.  Each segment leaves an unnormalised
 // partial (O, running max m, running sum l) in the workspace; the combine kernel merges
 // them with their log-sum-exp weights.
 //
-// Per CTA (192 threads): warp 0 loads (TMA for dense/paged rows and q~, 16-byte async
-// copies for indexed rows), warp 1 issues tcgen05 MMAs, warps 2-5 run the softmax and
-// the epilogue.  The 64 query rows (heads) of one query sit on the MMA N side and the
-// 128 cache rows of a tile on the M side:
+// Per CTA (320 threads): warp 0 loads (TMA for dense/paged rows and q~, 16-byte async
+// copies for indexed rows), warp 1 issues tcgen05 MMAs, warps 2-9 run the softmax and
+// the epilogue as two warpgroups of 32 head columns each.  The 64 query rows (heads) of
+// one query sit on the MMA N side and the 128 cache rows of a tile on the M side:
 //   S^T[tile rows, heads]  = C_tile (128 x 512, K-major)  *  Q~^T          (TMEM, fp32)
 //   O^T[latent, heads]    += C_tile^T (512 x 128, MN-major) * P^T          (TMEM, fp32)
 // so the latent dimension of O lives in TMEM lanes (4 blocks x 64 columns) and one
-// softmax thread owns one cache row of the tile.
+// softmax thread owns one cache row of the tile and 32 heads.  A tile stays in shared
+// memory from its score GEMM to its value GEMM, so every cache byte is read once.
 #include <math.h>
 
 #include <algorithm>
@@ -35,7 +36,8 @@ constexpr int kChunks = kLatent / 64;           // latent split in 128-byte swiz
 constexpr int kChunkBytes = kTile * 64 * 2;     // 16 KB: 128 rows x 64 latent
 constexpr int kQtChunkBytes = kRows * 64 * 2;   // 8 KB: 64 heads x 64 latent
 constexpr int kPBytes = kTile * kRows * 2;      // 16 KB: P^T, 128 rows x 64 heads (bf16)
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer, MMA, 8 softmax warps
+constexpr int kSoftmaxWarps = 8;
 constexpr float kTau = 8.0f;  // lazy rescale: the running max is raised only when a score
                               // exceeds it by more than 2^8 (probabilities stay <= 256)
 
@@ -166,6 +168,9 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, const 
 }
 
 // ------------------------------------------------------------------ producer (warp 0)
+// Streams, per segment, q~ (64 heads x 512) once and then every tile's 8 latent chunks
+// into the 8-slot ring; slot c of tile t is refilled once the value GEMM of tile t-1 has
+// consumed chunk c.
 template <int kMode>
 __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUtensorMap *tm_cache,
                               const CUtensorMap *tm_qt, int iq, long long t0, long long t1, int lane) {
@@ -219,32 +224,30 @@ __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUt
           cp_async_arrive_noinc(&bar[kBarCFull + c]);
         }
       } else {
-        if (lane == 0) {
-          const int j0 = t * kTile;
-          long long row[2] = {0, 0};
-          bool load[2];
+        const int j0 = t * kTile;
+        long long row[2] = {0, 0};
+        bool load[2];
 #pragma unroll
-          for (int hb = 0; hb < 2; ++hb) {
-            const int j = j0 + hb * 64;
-            load[hb] = j < sg.rows;
-            if (load[hb]) {
-              if constexpr (kMode == kModePaged) {
-                bool bad = false;
-                row[hb] = paged_row(p.page_table, b, j, p.max_pages, p.num_pages, bad);
-                if (bad) report_status(p.status, kStatusIndex);
-              } else {
-                row[hb] = dense_row(b, j, p.Lmax);
-              }
+        for (int hb = 0; hb < 2; ++hb) {
+          const int jj = j0 + hb * 64;
+          load[hb] = jj < sg.rows;
+          if (load[hb]) {
+            if constexpr (kMode == kModePaged) {
+              bool bad = false;
+              row[hb] = paged_row(p.page_table, b, jj, p.max_pages, p.num_pages, bad);
+              if (bad) report_status(p.status, kStatusIndex);
+            } else {
+              row[hb] = dense_row(b, jj, p.Lmax);
             }
           }
-          const uint32_t bytes = (load[0] ? 8192u : 0u) + (load[1] ? 8192u : 0u);
-          for (int c = 0; c < kChunks; ++c) {
-            if (!mbar_wait(&bar[kBarCEmpty + c], (tile_k & 1) ^ 1, sh.abort_flag, p.status)) return;
-            mbar_arrive_expect_tx(&bar[kBarCFull + c], bytes);
+        }
+        const uint32_t bytes = (load[0] ? 8192u : 0u) + (load[1] ? 8192u : 0u);
+        for (int c = 0; c < kChunks; ++c) {
+          if (!mbar_wait(&bar[kBarCEmpty + c], (tile_k & 1) ^ 1, sh.abort_flag, p.status)) return;
+          mbar_arrive_expect_tx(&bar[kBarCFull + c], bytes);
 #pragma unroll
-            for (int hb = 0; hb < 2; ++hb)
-              if (load[hb]) tma_load_2d(sh.chunk(c) + hb * 8192, tm_cache, &bar[kBarCFull + c], c * 64, (int)row[hb]);
-          }
+          for (int hb = 0; hb < 2; ++hb)
+            if (load[hb]) tma_load_2d(sh.chunk(c) + hb * 8192, tm_cache, &bar[kBarCFull + c], c * 64, (int)row[hb]);
         }
       }
     }
@@ -252,6 +255,19 @@ __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUt
 }
 
 // ------------------------------------------------------------------ MMA issuer (warp 1)
+// Rows past the end of the sequence may hold any bits: zero them in the landed chunk so
+// that a masked (zero) probability never meets a NaN or Inf in the value product.
+template <int kMode>
+__device__ __forceinline__ void prepare_chunk(uint32_t cbase, int n_valid, int lane) {
+  if (kMode != kModeIndexed && n_valid < kTile) {
+    for (int idx = lane; idx < (kTile - n_valid) * 8; idx += 32)
+      st_shared_v4(cbase + (n_valid + idx / 8) * 128 + (idx % 8) * 16, 0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
+  if (kMode == kModeIndexed) fence_proxy_async_smem();  // rows written by 16-byte async copies
+  __syncwarp();
+}
+
 template <int kMode>
 __device__ void mma_role(const AttendParams &p, const Shared &sh, uint32_t tmem, long long t0, long long t1,
                          int lane) {
@@ -268,22 +284,14 @@ __device__ void mma_role(const AttendParams &p, const Shared &sh, uint32_t tmem,
     if (!wait_warp(&bar[kBarQFull], q_use & 1, sh, p.status)) return;
     ++q_use;
     for (int t = sg.lo; t < sg.hi; ++t, ++tile_k) {
+      const int n_valid = min(kTile, sg.rows - t * kTile);
+      // S^T[tile rows, heads] = C_tile * Q~^T, K = 512 latent in 8 chunks of 4 MMA steps
       const uint32_t sb = s_use & 1;
       if (!wait_warp(&bar[kBarSEmpty + sb], ((s_use >> 1) & 1) ^ 1, sh, p.status)) return;
       tc_fence_after();
-      const int n_valid = min(kTile, sg.rows - t * kTile);
       for (int c = 0; c < kChunks; ++c) {
         if (!wait_warp(&bar[kBarCFull + c], tile_k & 1, sh, p.status)) return;
-        if (kMode != kModeIndexed && n_valid < kTile) {
-          // rows past the end of the sequence may hold any bits: zero them so that a
-          // masked (zero) probability never meets a NaN or Inf in the value product
-          const uint32_t cbase = c_base + c * kChunkBytes;
-          for (int idx = lane; idx < (kTile - n_valid) * 8; idx += 32)
-            st_shared_v4(cbase + (n_valid + idx / 8) * 128 + (idx % 8) * 16, 0u, 0u, 0u, 0u);
-          fence_proxy_async_smem();
-        }
-        if (kMode == kModeIndexed) fence_proxy_async_smem();
-        __syncwarp();
+        prepare_chunk<kMode>(c_base + c * kChunkBytes, n_valid, lane);
         tc_fence_after();
         if (lane == 0) {
 #pragma unroll
@@ -300,6 +308,7 @@ __device__ void mma_role(const AttendParams &p, const Shared &sh, uint32_t tmem,
         if (t == sg.hi - 1) umma_commit(&bar[kBarQEmpty]);
       }
       ++s_use;
+      // O^T[latent, heads] += C_tile^T * P^T, four 128-lane latent blocks, K = 128 rows
       if (!wait_warp(&bar[kBarPFull], p_use & 1, sh, p.status)) return;
       ++p_use;
       if (t == sg.lo && !wait_warp(&bar[kBarOEmpty], (o_use & 1) ^ 1, sh, p.status)) return;
@@ -328,124 +337,118 @@ __device__ void mma_role(const AttendParams &p, const Shared &sh, uint32_t tmem,
   }
 }
 
-// ------------------------------------------------------------------ softmax + epilogue (warps 2-5)
-// Thread `row` owns cache row `row` of the tile and all 64 head columns of S^T; the 64
-// columns are handled in two halves of 32 to keep the registers within budget.
+// ------------------------------------------------------------------ softmax + epilogue (warps 2-9)
+// Two warpgroups; warpgroup wg owns head columns [32 wg, 32 wg + 32) of S^T and O^T.  Thread
+// `row` of a warpgroup owns cache row `row` of the tile.  The running max per column lives
+// in shared memory (read with broadcast loads).  With 10 warps, three share an SM
+// sub-partition's register file, which caps a thread at 168 registers.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int kMode>
 __device__ void softmax_role(const AttendParams &p, const Shared &sh, uint32_t tmem, int g, int iq, long long t0,
                              long long t1, int warp, int lane) {
   uint64_t *bar = sh.bar;
-  const int wq = warp & 3;                 // TMEM lane quadrant of this warp
-  const int tid = (warp - 2) * 32 + lane;  // 0..127 within the softmax group
-  const int row = wq * 32 + lane;          // tile row (TMEM lane) owned by this thread
+  const int wg = (warp - 2) >> 2;              // warpgroup: head columns [32 wg, 32 wg + 32)
+  const int wq = warp & 3;                     // TMEM lane quadrant of this warp
+  const int tid = ((warp - 2) & 3) * 32 + lane;  // 0..127 within the warpgroup
+  const int row = wq * 32 + lane;              // tile row (TMEM lane) owned by this thread
+  const uint32_t bar_id = 1 + wg;
+  const int col0 = wg * 32;
   const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
   const uint32_t p_row = smem_u32(sh.pbuf()) + row * 128;
-  float *red = sh.red;
-  float *m_used = sh.m_used;
-  float *alpha = sh.alpha;
+  float *red = sh.red;          // [4 quadrants][64 columns]
+  float *m_used = sh.m_used;    // [64]
+  float *alpha = sh.alpha;      // [64]
   uint32_t s_use = 0, p_use = 0, o_use = 0;
-  if (tid < kRows) {
-    m_used[tid] = -INFINITY;
-    alpha[tid] = 1.f;
-  }
-  named_bar_sync(1, 128);
+  const float *mu = m_used + col0;  // running max of this warpgroup's columns (log2 units)
+  if (tid < 32) m_used[col0 + tid] = -INFINITY;
+  named_bar_sync(bar_id, 128);
   SegIter it(t0, t1);
   Seg sg;
   while (it.next(p, kMode, sg)) {
     const int qi = (kMode == kModeIndexed) ? sg.s % p.Q : iq;
     // positions of this CTA's query that are visible: dense/paged rows 0..L_b-Q+qi, or the list
     const int n_vis = (kMode == kModeIndexed) ? p.K : sg.rows - p.Q + qi + 1;
-    float l_part[kRows];
+    float l_part[32];
 #pragma unroll
-    for (int c = 0; c < kRows; ++c) l_part[c] = 0.f;
+    for (int c = 0; c < 32; ++c) l_part[c] = 0.f;
     for (int t = sg.lo; t < sg.hi; ++t) {
       const uint32_t sb = s_use & 1;
       mbar_wait(&bar[kBarSFull + sb], (s_use >> 1) & 1, sh.abort_flag, p.status);
+      tc_fence_after();
+      const bool valid = (t * kTile + row) < n_vis;
+      float s2[32];
+      {
+        uint32_t r[32];
+        tmem_ld32(t_lane + kTmemS + sb * kRows + col0, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) s2[c] = valid ? __uint_as_float(r[c]) * p.scale_log2 : -INFINITY;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[kBarSEmpty + sb]);
+      ++s_use;
+      bool flag = false;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) flag |= s2[c] > mu[c] + kTau;
+      const bool any = named_bar_or(bar_id, 128, flag);
+      if (*sh.abort_flag) return;
+      if (any) {
+        // new running max for this warpgroup's 32 columns
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float mx = warp_max_f32(s2[c]);
+          if (lane == c) red[wq * kRows + col0 + c] = mx;
+        }
+        named_bar_sync(bar_id, 128);
+        if (tid < 32) {
+          const int c = col0 + tid;
+          const float mt = fmaxf(fmaxf(red[c], red[kRows + c]), fmaxf(red[2 * kRows + c], red[3 * kRows + c]));
+          const float mo = m_used[c];
+          const float mn = fmaxf(mo, mt);
+          alpha[c] = (mn == -INFINITY) ? 1.f : fast_exp2(mo - mn);
+          m_used[c] = mn;
+        }
+        named_bar_sync(bar_id, 128);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) l_part[c] *= alpha[col0 + c];
+      }
       // the P buffer is free and the previous value product has finished
       mbar_wait(&bar[kBarPEmpty], (p_use & 1) ^ 1, sh.abort_flag, p.status);
       tc_fence_after();
-      const bool valid = (t * kTile + row) < n_vis;
-      bool any_tile = false;
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float s2[32];
-        {
+      if (any && t > sg.lo) {
+        // running max moved: rescale this warpgroup's O^T columns in TMEM
+#pragma unroll 1
+        for (int mb = 0; mb < 4; ++mb) {
           uint32_t r[32];
-          tmem_ld32(t_lane + kTmemS + sb * kRows + hf * 32, r);
+          const uint32_t addr = t_lane + kTmemO + mb * kRows + col0;
+          tmem_ld32(addr, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) s2[c] = valid ? __uint_as_float(r[c]) * p.scale_log2 : -INFINITY;
+          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha[col0 + j]);
+          tmem_st32(addr, r);
         }
-        if (hf == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bar[kBarSEmpty + sb]);
-        }
-        bool flag = false;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) flag |= s2[c] > m_used[hf * 32 + c] + kTau;
-        const bool any = named_bar_or(1, 128, flag);
-        if (*sh.abort_flag) return;
-        if (any) {
-          // new running max for these 32 columns
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float mx = warp_max_f32(s2[c]);
-            if (lane == c) red[wq * kRows + hf * 32 + c] = mx;
-          }
-          named_bar_sync(1, 128);
-          if (tid < 32) {
-            const int c = hf * 32 + tid;
-            const float mt =
-                fmaxf(fmaxf(red[c], red[kRows + c]), fmaxf(red[2 * kRows + c], red[3 * kRows + c]));
-            const float mo = m_used[c];
-            const float mn = fmaxf(mo, mt);
-            alpha[c] = (mn == -INFINITY) ? 1.f : exp2f(mo - mn);
-            m_used[c] = mn;
-          }
-          named_bar_sync(1, 128);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) l_part[hf * 32 + c] *= alpha[hf * 32 + c];
-          any_tile = true;
-        }
-        // probabilities, rounded to bf16 for the value product; l sums the rounded values
-#pragma unroll
-        for (int pc = 0; pc < 4; ++pc) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c0 = pc * 8 + 2 * e;
-            const float m0 = m_used[hf * 32 + c0], m1 = m_used[hf * 32 + c0 + 1];
-            const float p0 = (s2[c0] == -INFINITY) ? 0.f : exp2f(s2[c0] - m0);
-            const float p1 = (s2[c0 + 1] == -INFINITY) ? 0.f : exp2f(s2[c0 + 1] - m1);
-            w[e] = pack_bf16x2(p0, p1);
-            l_part[hf * 32 + c0] += bf16lo_to_f32(w[e]);
-            l_part[hf * 32 + c0 + 1] += bf16hi_to_f32(w[e]);
-          }
-          st_shared_v4(p_row + (((hf * 4 + pc) ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);
-        }
+        tmem_st_wait();
       }
-      ++s_use;
-      if (any_tile) {
-        if (t > sg.lo) {
-          // running max moved: rescale the partial O^T columns (heads) in TMEM
-#pragma unroll 1
-          for (int mb = 0; mb < 4; ++mb) {
+      // probabilities, rounded to bf16 for the value product; l sums the rounded values
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-              uint32_t r[32];
-              const uint32_t addr = t_lane + kTmemO + mb * kRows + hf * 32;
-              tmem_ld32(addr, r);
-              tmem_ld_wait();
+      for (int pc = 0; pc < 4; ++pc) {
+        uint32_t w[4];
 #pragma unroll
-              for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha[hf * 32 + j]);
-              tmem_st32(addr, r);
-            }
-          }
-          tmem_st_wait();
+        for (int e = 0; e < 4; ++e) {
+          const int c0 = pc * 8 + 2 * e;
+          const float p0 = (s2[c0] == -INFINITY) ? 0.f : fast_exp2(s2[c0] - mu[c0]);
+          const float p1 = (s2[c0 + 1] == -INFINITY) ? 0.f : fast_exp2(s2[c0 + 1] - mu[c0 + 1]);
+          w[e] = pack_bf16x2(p0, p1);
+          l_part[c0] += bf16lo_to_f32(w[e]);
+          l_part[c0 + 1] += bf16hi_to_f32(w[e]);
         }
-        named_bar_sync(1, 128);
-        if (tid < kRows) alpha[tid] = 1.f;
+        st_shared_v4(p_row + (((wg * 4 + pc) ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -457,41 +460,38 @@ __device__ void softmax_role(const AttendParams &p, const Shared &sh, uint32_t t
     mbar_wait(&bar[kBarOFull], o_use & 1, sh.abort_flag, p.status);
     tc_fence_after();
 #pragma unroll
-    for (int c = 0; c < kRows; ++c) {
+    for (int c = 0; c < 32; ++c) {
       float v = l_part[c];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == (c & 31)) red[wq * kRows + c] = v;
+      if (lane == c) red[wq * kRows + col0 + c] = v;
     }
-    named_bar_sync(1, 128);
+    named_bar_sync(bar_id, 128);
     if (*sh.abort_flag) return;
     const long long slot =
         (kMode == kModeIndexed) ? (long long)g + sg.s : ((long long)g + sg.s) * p.Q + iq;
-    if (tid < kRows) {
-      const int c = tid;
+    if (tid < 32) {
+      const int c = col0 + tid;
       p.part_m[slot * kRows + c] = m_used[c];
       p.part_l[slot * kRows + c] = red[c] + red[kRows + c] + red[2 * kRows + c] + red[3 * kRows + c];
     }
     float *po = p.part_o + slot * kRows * kLatent;
 #pragma unroll 1
     for (int mb = 0; mb < 4; ++mb) {
+      uint32_t r[32];
+      tmem_ld32(t_lane + kTmemO + mb * kRows + col0, r);
+      tmem_ld_wait();
+      const int lat = mb * 128 + wq * 32 + lane;
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t r[32];
-        tmem_ld32(t_lane + kTmemO + mb * kRows + hf * 32, r);
-        tmem_ld_wait();
-        const int lat = mb * 128 + wq * 32 + lane;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) po[(hf * 32 + j) * kLatent + lat] = __uint_as_float(r[j]);
-      }
+      for (int j = 0; j < 32; ++j) po[(col0 + j) * kLatent + lat] = __uint_as_float(r[j]);
     }
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[kBarOEmpty]);
     ++o_use;
-    named_bar_sync(1, 128);
-    if (tid < kRows) m_used[tid] = -INFINITY;
-    named_bar_sync(1, 128);
+    named_bar_sync(bar_id, 128);
+    if (tid < 32) m_used[col0 + tid] = -INFINITY;
+    named_bar_sync(bar_id, 128);
   }
 }
 
@@ -524,12 +524,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sh.bar[kBarQEmpty], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sh.bar[kBarSFull + i], 1);
-      mbar_init(&sh.bar[kBarSEmpty + i], 4);
+      mbar_init(&sh.bar[kBarSEmpty + i], kSoftmaxWarps);
     }
-    mbar_init(&sh.bar[kBarPFull], 4);
+    mbar_init(&sh.bar[kBarPFull], kSoftmaxWarps);
     mbar_init(&sh.bar[kBarPEmpty], 1);
     mbar_init(&sh.bar[kBarOFull], 1);
-    mbar_init(&sh.bar[kBarOEmpty], 4);
+    mbar_init(&sh.bar[kBarOEmpty], kSoftmaxWarps);
     *sh.abort_flag = 0;
     fence_barrier_init();
   }
@@ -579,17 +579,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ combine
-// One block per (sequence b, query i) and group of 4 heads; thread t owns latent 4t..4t+3.
+// One block per (sequence b, query i) and pair of heads; thread t owns latent 4t..4t+3.
+// The partial of every CTA group that processed tiles of b is weighted by
+// 2^(m_g - M) (M the largest running max) and the weighted sums are normalised.
+constexpr int kCombineHeads = 2;
+constexpr int kMaxSlotsPerSeq = 1024;
+
 __global__ void __launch_bounds__(128) combine_kernel(const AttendParams p, int mode) {
   const int v = blockIdx.x;  // b * Q + i
   const int b = v / p.Q, i = v % p.Q;
   const int s = (mode == kModeIndexed) ? v : b;
   __shared__ long long sh_info[3];
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
+  __shared__ float sh_w[kCombineHeads][kMaxSlotsPerSeq];
+  __shared__ float sh_l[kCombineHeads][kMaxSlotsPerSeq];
+  __shared__ float sh_norm[kCombineHeads][2];  // 1/den, lse
+  const int tid = threadIdx.x;
+  if (tid < 32) {
     const int ns = num_seqs(p, mode);
     long long before = 0, total = 0;
-    for (int x = lane; x < ns; x += 32) {
+    for (int x = tid; x < ns; x += 32) {
       const int nt = seq_tiles(p, mode, x);
       total += nt;
       if (x < s) before += nt;
@@ -599,7 +607,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const AttendParams p, int 
       before += __shfl_xor_sync(0xffffffffu, before, o);
       total += __shfl_xor_sync(0xffffffffu, total, o);
     }
-    if (lane == 0) {
+    if (tid == 0) {
       sh_info[0] = before;
       sh_info[1] = seq_tiles(p, mode, s);
       sh_info[2] = total;
@@ -612,45 +620,67 @@ __global__ void __launch_bounds__(128) combine_kernel(const AttendParams p, int 
   }
   __syncthreads();
   const long long ts = sh_info[0], nt = sh_info[1], T = sh_info[2], G = p.groups;
-  const int lat = threadIdx.x * 4;
-  for (int hh = 0; hh < 4; ++hh) {
-    const int h = blockIdx.y * 4 + hh;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    float M = -INFINITY, den = 0.f;
-    if (nt > 0) {
-      const long long g_first = ((ts + 1) * G - 1) / T;
-      const long long g_last = ((ts + nt) * G - 1) / T;
-      for (long long gg = g_first; gg <= g_last; ++gg) {
-        if (group_start(gg, T, G) >= group_start(gg + 1, T, G)) continue;
-        const long long slot = (mode == kModeIndexed) ? gg + s : (gg + s) * p.Q + i;
-        M = fmaxf(M, p.part_m[slot * kRows + h]);
-      }
-      if (M != -INFINITY) {
-        for (long long gg = g_first; gg <= g_last; ++gg) {
-          if (group_start(gg, T, G) >= group_start(gg + 1, T, G)) continue;
-          const long long slot = (mode == kModeIndexed) ? gg + s : (gg + s) * p.Q + i;
-          const float m = p.part_m[slot * kRows + h];
-          if (m == -INFINITY) continue;
-          const float w = exp2f(m - M);
-          den += w * p.part_l[slot * kRows + h];
-          const float4 o = *reinterpret_cast<const float4 *>(p.part_o + (slot * kRows + h) * kLatent + lat);
-          acc[0] += w * o.x;
-          acc[1] += w * o.y;
-          acc[2] += w * o.z;
-          acc[3] += w * o.w;
-        }
+  long long g_first = 0, g_last = -1;
+  if (nt > 0) {
+    g_first = ((ts + 1) * G - 1) / T;
+    g_last = ((ts + nt) * G - 1) / T;
+  }
+  const int nslot = (int)min(g_last - g_first + 1, (long long)kMaxSlotsPerSeq);
+  auto slot_of = [&](long long gg) -> long long {
+    return (mode == kModeIndexed) ? gg + s : (gg + s) * p.Q + i;
+  };
+  const int h0 = blockIdx.y * kCombineHeads;
+  // weights: running maxima of the non-empty groups, then 2^(m - M) and the normaliser
+  for (int x = tid; x < kCombineHeads * nslot; x += 128) {
+    const int hh = x / nslot, k = x % nslot;
+    const long long gg = g_first + k;
+    float m = -INFINITY, l = 0.f;
+    if (group_start(gg, T, G) < group_start(gg + 1, T, G)) {
+      m = p.part_m[slot_of(gg) * kRows + h0 + hh];
+      l = p.part_l[slot_of(gg) * kRows + h0 + hh];
+    }
+    sh_w[hh][k] = m;
+    sh_l[hh][k] = l;
+  }
+  __syncthreads();
+  if (tid < kCombineHeads) {
+    const int hh = tid;
+    float M = -INFINITY;
+    for (int k = 0; k < nslot; ++k) M = fmaxf(M, sh_w[hh][k]);
+    float den = 0.f;
+    for (int k = 0; k < nslot; ++k) {
+      const float m = sh_w[hh][k];
+      const float w = (m == -INFINITY) ? 0.f : exp2f(m - M);
+      sh_w[hh][k] = w;
+      den += w * sh_l[hh][k];
+    }
+    const bool ok = (M != -INFINITY) && den > 0.f;
+    sh_norm[hh][0] = ok ? 1.f / den : 0.f;
+    sh_norm[hh][1] = ok ? (M + log2f(den)) * 0.69314718055994530942f : -INFINITY;
+  }
+  __syncthreads();
+  const int lat = tid * 4;
+#pragma unroll
+  for (int hh = 0; hh < kCombineHeads; ++hh) {
+    const int h = h0 + hh;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int k = 0; k < nslot; ++k) {
+      const float w = sh_w[hh][k];
+      if (w != 0.f) {
+        const float4 o = *reinterpret_cast<const float4 *>(p.part_o + (slot_of(g_first + k) * kRows + h) * kLatent + lat);
+        acc.x += w * o.x;
+        acc.y += w * o.y;
+        acc.z += w * o.z;
+        acc.w += w * o.w;
       }
     }
-    uint2 outv = make_uint2(0u, 0u);
-    float lse = -INFINITY;
-    if (M != -INFINITY && den > 0.f) {
-      const float inv = 1.f / den;
-      outv.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-      outv.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-      lse = (M + log2f(den)) * 0.69314718055994530942f;
-    }
+    const float inv = sh_norm[hh][0];
+    uint2 outv;
+    outv.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    outv.y = pack_bf16x2(acc.z * inv, acc.w * inv);
     *reinterpret_cast<uint2 *>(p.o_latent + ((long long)v * kRows + h) * kLatent + lat) = outv;
-    if (p.lse != nullptr && threadIdx.x == 0) p.lse[(long long)v * kRows + h] = lse;
+    if (p.lse != nullptr && tid == 0) p.lse[(long long)v * kRows + h] = sh_norm[hh][1];
   }
 }
 
@@ -710,7 +740,7 @@ static cudaError_t launch_attend_mode(const CUtensorMap &tm_cache, const CUtenso
   attend::attend_kernel<kMode><<<grid, attend::kThreads, attend::kSmemBytes, stream>>>(tm_cache, tm_qt, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dim3 cgrid(p.B * p.Q, kHeads / 4);
+  dim3 cgrid(p.B * p.Q, kHeads / attend::kCombineHeads);
   attend::combine_kernel<<<cgrid, 128, 0, stream>>>(p, kMode);
   return cudaGetLastError();
 }

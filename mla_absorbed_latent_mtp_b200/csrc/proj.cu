@@ -5,8 +5,9 @@
 // side (128 rows per CTA) and the tokens on N:
 //   D[m, n] = A_h[m, k] * X[n, h, k]^T,   A_h = W_UK[h]^T (MN-major) or W_UV[h] (K-major).
 // One CTA per (head, 128-row weight block, token tile): warp 0 streams 64-wide K chunks
-// through a 4-stage TMA ring, warp 1 issues tcgen05 MMAs into TMEM, warps 2-5 convert the
-// fp32 accumulator to bf16 and store it.
+// through a TMA ring, warp 1 issues tcgen05 MMAs into TMEM, warps 2-5 convert the
+// fp32 accumulator to bf16 and store it.  All K chunks of the weight block are in flight
+// at once when shared memory allows (up to 8 stages).
 #include <algorithm>
 
 #include "internal.h"
@@ -16,21 +17,20 @@ namespace mla {
 namespace proj {
 
 constexpr int kThreads = 192;
-constexpr int kStages = 4;
+constexpr int kMaxStages = 8;
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kMaxNT = 128;
-constexpr int kABytes = kBM * kBK * 2;      // 16 KB per stage
-constexpr int kBBytesMax = kMaxNT * kBK * 2; // 16 KB per stage
-constexpr int kOffA = 0;
-constexpr int kOffB = kOffA + kStages * kABytes;
-constexpr int kOffBar = kOffB + kStages * kBBytesMax;
-constexpr int kOffMisc = kOffBar + (2 * kStages + 1) * 8;
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+constexpr int kABytes = kBM * kBK * 2;  // 16 KB per stage
 constexpr uint32_t kTmemCols = 128;
+constexpr int kSmemLimit = 227 * 1024;
+
+// Shared memory: `stages` A tiles (16 KB), `stages` B tiles (n_tile x 128 B), barriers.
+__host__ __device__ constexpr int smem_bytes(int stages, int n_tile) {
+  return stages * (kABytes + n_tile * kBK * 2) + (2 * kMaxStages + 1) * 8 + 16 + 1024;
+}
 
 struct Params {
-  int n, H, M_total, K_total, n_tile;
+  int n, H, M_total, K_total, n_tile, stages;
   uint16_t *out;
 };
 
@@ -39,11 +39,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     proj_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(base + kOffBar);
-  uint64_t *empty = full + kStages;
-  uint64_t *done = empty + kStages;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kOffMisc);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(base + kOffMisc + 4);
+  const int kStages = p.stages;
+  const int b_bytes = p.n_tile * kBK * 2;
+  uint8_t *a_stage0 = base;
+  uint8_t *b_stage0 = base + kStages * kABytes;
+  uint64_t *full = reinterpret_cast<uint64_t *>(b_stage0 + kStages * b_bytes);
+  uint64_t *empty = full + kMaxStages;
+  uint64_t *done = empty + kMaxStages;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int h = blockIdx.x, mb = blockIdx.y, nt = blockIdx.z;
@@ -76,7 +80,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = kc % kStages, use = kc / kStages;
         if (!mbar_wait(&empty[s], (use & 1) ^ 1, abort_flag, nullptr)) break;
         mbar_arrive_expect_tx(&full[s], kABytes + NT * kBK * 2);
-        uint8_t *a_dst = base + kOffA + s * kABytes;
+        uint8_t *a_dst = a_stage0 + s * kABytes;
         if (kAMajorMN) {
           // W_UK[h][d][r]: box {64 r, 64 d}; two boxes cover the 128 r of this block
           tma_load_3d(a_dst, &tm_w, &full[s], mb * kBM, kc * kBK, h);
@@ -85,7 +89,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // W_UV[h][d][r]: box {64 r, 128 d}
           tma_load_3d(a_dst, &tm_w, &full[s], kc * kBK, mb * kBM, h);
         }
-        tma_load_3d(base + kOffB + s * kBBytesMax, &tm_x, &full[s], kc * kBK, h, nt * NT);
+        tma_load_3d(b_stage0 + s * b_bytes, &tm_x, &full[s], kc * kBK, h, nt * NT);
       }
     }
   } else if (warp == 1) {
@@ -97,8 +101,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t a_base = smem_u32(base + kOffA + s * kABytes);
-        const uint32_t b_base = smem_u32(base + kOffB + s * kBBytesMax);
+        const uint32_t a_base = smem_u32(a_stage0 + s * kABytes);
+        const uint32_t b_base = smem_u32(b_stage0 + s * b_bytes);
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
           // MN-major A: 64-wide r atoms 8 KB apart (LBO), 8-row d groups 1 KB apart (SBO);
@@ -154,18 +158,21 @@ static cudaError_t launch_proj_t(const CUtensorMap &tm_w, const CUtensorMap &tm_
   cudaGetDevice(&dev);
   if (configured_device != dev) {
     cudaError_t e = cudaFuncSetAttribute(proj::proj_kernel<kAMajorMN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         proj::kSmemBytes);
+                                         proj::kSmemLimit);
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
   dim3 grid(p.H, p.M_total / proj::kBM, (p.n + p.n_tile - 1) / p.n_tile);
-  proj::proj_kernel<kAMajorMN><<<grid, proj::kThreads, proj::kSmemBytes, stream>>>(tm_w, tm_x, p);
+  proj::proj_kernel<kAMajorMN><<<grid, proj::kThreads, proj::smem_bytes(p.stages, p.n_tile), stream>>>(tm_w, tm_x, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_proj(bool a_mn_major, const CUtensorMap &tm_w, const CUtensorMap &tm_x, int n, int H,
                         int M_total, int K_total, int n_tile, uint16_t *out, cudaStream_t stream) {
-  proj::Params p{n, H, M_total, K_total, n_tile, out};
+  // keep every K chunk of the weight block in flight when it fits
+  int stages = std::min(proj::kMaxStages, K_total / proj::kBK);
+  while (stages > 2 && proj::smem_bytes(stages, n_tile) > proj::kSmemLimit) --stages;
+  proj::Params p{n, H, M_total, K_total, n_tile, stages, out};
   return a_mn_major ? launch_proj_t<true>(tm_w, tm_x, p, stream) : launch_proj_t<false>(tm_w, tm_x, p, stream);
 }
 
