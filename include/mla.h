@@ -123,6 +123,26 @@ mla_status mla_up_proj(const uint16_t *o_latent, const uint16_t *w_uv, uint16_t 
                        int n, int H, int D, int R, void *stream);
 
 /*
+ * mla_attend_dense for callers that cannot allocate device memory (for example a plugin
+ * inside a host runtime that owns all device memory and passes its plugins no workspace,
+ * or a runtime whose memory plan is fixed at start-up).  There is no counterpart on the
+ * pages: it is a packaging variant of mla_attend_dense, with the same arguments minus
+ * the workspace and the same results.
+ *  - Scratch comes from a 32 MiB array inside the library, held by every GPU that loads
+ *    the library until the process exits.  Sizes whose mla_attend_workspace_bytes(B, Q, H, R)
+ *    exceeds 32 MiB return MLA_ERR_WORKSPACE and enqueue nothing.
+ *  - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *    with that device current; make that first call before any stream capture.
+ *  - All calls share the one array, so calls whose kernels overlap on the GPU (different
+ *    streams, or several host threads) race and corrupt each other's results; serialise
+ *    them.  No part of the array has to start at zero.
+ */
+mla_status mla_attend_dense_noalloc(const uint16_t *q_tilde, const uint16_t *cache, const int32_t *seq_lens,
+                                    int B, int Q, int H, int R, int Lmax, float scale, uint16_t *o_latent,
+                                    float *lse, int32_t *status, void *stream);
+
+/*
  * Bytes of workspace the mla_attend_* calls need for B sequences of Q queries on the
  * current device (split-L partial results and their max/sum terms).  0 on bad sizes.
  */

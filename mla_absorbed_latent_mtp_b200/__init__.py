@@ -20,7 +20,7 @@ H, D, R, PAGE = 64, 256, 512, 64
 SCALE = 1.0 / 16.0
 
 EXPORTS = ("mla_status_string", "mla_last_error_string", "mla_absorb_q", "mla_attend_dense", "mla_attend_paged", "mla_attend_indexed",
-           "mla_up_proj", "mla_attend_workspace_bytes", "mla_debug_gather")
+           "mla_up_proj", "mla_attend_workspace_bytes", "mla_debug_gather", "mla_attend_dense_noalloc")
 
 
 class MLAError(RuntimeError):
@@ -54,8 +54,9 @@ def lib():
     L.mla_attend_workspace_bytes.argtypes = [i32, i32, i32, i32]
     L.mla_attend_workspace_bytes.restype = sz
     L.mla_debug_gather.argtypes = [i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp]
+    L.mla_attend_dense_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp, vp, vp]
     for name in ("mla_absorb_q", "mla_up_proj", "mla_attend_dense", "mla_attend_paged", "mla_attend_indexed",
-                 "mla_debug_gather"):
+                 "mla_debug_gather", "mla_attend_dense_noalloc"):
         getattr(L, name).restype = ctypes.c_int32
     _lib = L
     return L
@@ -142,6 +143,19 @@ def mla_attend_dense(q_tilde, cache, seq_lens=None, scale=SCALE, workspace=None,
     _check("mla_attend_dense", lib().mla_attend_dense(
         _ptr(q_tilde), _ptr(cache), _ptr(seq_lens), B, Q, H, R, Lmax, scale, _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(o_latent), _ptr(lse), _ptr(status), _stream(stream)))
+    return o_latent, lse
+
+
+def mla_attend_dense_noalloc(q_tilde, cache, seq_lens=None, scale=SCALE, o_latent=None, lse=None, status=None,
+                             want_lse=True, stream=None):
+    """mla_attend_dense without a workspace argument: for callers that cannot allocate
+    device memory, the scratch is a fixed 32 MiB array inside the library (see mla.h)."""
+    _check_cuda(q_tilde, cache, seq_lens, o_latent, lse, status)
+    B, Q = q_tilde.shape[0], q_tilde.shape[1]
+    o_latent, lse = _attend_outputs(q_tilde, o_latent, lse, want_lse)
+    _check("mla_attend_dense_noalloc", lib().mla_attend_dense_noalloc(
+        _ptr(q_tilde), _ptr(cache), _ptr(seq_lens), B, Q, H, R, cache.shape[1], scale, _ptr(o_latent), _ptr(lse),
+        _ptr(status), _stream(stream)))
     return o_latent, lse
 
 

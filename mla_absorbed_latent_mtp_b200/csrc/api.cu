@@ -68,6 +68,8 @@ static mla_status cuda_status(cudaError_t e) {
   return MLA_ERR_CUDA;
 }
 
+mla_status record_cuda_error(cudaError_t e) { return cuda_status(e); }
+
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;

@@ -53,5 +53,7 @@ cudaError_t launch_proj(bool a_mn_major, const CUtensorMap &tm_w, const CUtensor
                         int M_total, int K_total, int n_tile, uint16_t *out, cudaStream_t stream);
 
 int device_sm_count();
+// Records e as the calling thread's last CUDA error; returns MLA_ERR_CUDA (MLA_OK for success).
+int32_t record_cuda_error(cudaError_t e);
 
 }  // namespace mla
