@@ -379,7 +379,7 @@ def main(argv=None):
     stage = [sum(ev[k][j].elapsed_time(ev[k][j + 1]) for k in range(K)) / K for j in range(3)]
     ms, value = aggregate(local_ms, acc["total"], device)
     stage = reduce_max(stage, device)
-    launches = K * 4  # absorb, attend, combine, up-projection
+    launches = K * 4  # absorb, attend, split-L combine, up-projection
 
     # end to end through the public API with host buffers: H2D inputs, D2H output per step
     Ke = max(1, min(args.e2e_steps, K))
@@ -423,7 +423,7 @@ def main(argv=None):
                    "cache_rows": int(sum(int(x) for x in wl.seq_lens)) if wl.mode != "indexed" else None,
                    "heads": 64, "head_dim": 256, "latent": 512, "parallelism": f"dp{world} (independent batches)",
                    "l2": "inputs larger than L2 (cache %.0f MB per rank)" % (acc["cache"] / 1e6)},
-        "stages_ms": {"absorb_q": stage[0], "attend": stage[2 - 1], "up_proj": stage[2]},
+        "stages_ms": {"absorb_q": stage[0], "attend": stage[1], "up_proj": stage[2]},
         "attend_tflops": acc["flops_attend"] / (stage[1] * 1e-3) / 1e12,
         "roofline": roofline,
         "e2e": {"value": e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
