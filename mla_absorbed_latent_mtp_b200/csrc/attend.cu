@@ -2,7 +2,7 @@
 // original scale, softmax over the causally visible positions of section 4, value
 // sum kept in latent space) for a contiguous, paged or index-listed latent cache.
 //
-// Work decomposition.  Every sequence's visible rows are cut into 128-row tiles; the
+// Work decomposition.  Every sequence's visible rows are cut into 64-row tiles; the
 // tiles of all sequences form one list that G CTA groups split into equal contiguous
 // ranges (a range may cross sequence boundaries; each piece is a "segment").  A group
 // holds one CTA per query of a verify window (Q CTAs for dense/paged caches, all reading
@@ -11,15 +11,18 @@
 // partial (O, running max m, running sum l) in the workspace; the combine kernel merges
 // them with their log-sum-exp weights.
 //
-// Per CTA (320 threads): warp 0 loads (TMA for dense/paged rows and q~, 16-byte async
-// copies for indexed rows), warp 1 issues tcgen05 MMAs, warps 2-9 run the softmax and
-// the epilogue as two warpgroups of 32 head columns each.  The 64 query rows (heads) of
-// one query sit on the MMA N side and the 128 cache rows of a tile on the M side:
-//   S^T[tile rows, heads]  = C_tile (128 x 512, K-major)  *  Q~^T          (TMEM, fp32)
-//   O^T[latent, heads]    += C_tile^T (512 x 128, MN-major) * P^T          (TMEM, fp32)
-// so the latent dimension of O lives in TMEM lanes (4 blocks x 64 columns) and one
-// softmax thread owns one cache row of the tile and 32 heads.  A tile stays in shared
-// memory from its score GEMM to its value GEMM, so every cache byte is read once.
+// Per CTA (352 threads): warp 0 loads (TMA for dense/paged rows and q~, 16-byte async
+// copies for indexed rows), warp 1 issues the score MMAs and warp 10 the value MMAs
+// (tcgen05), warps 2-9 run the softmax and the epilogue as two warpgroups of 32 head
+// columns each.  The 64 query rows (heads) of
+// one query sit on the MMA N side and the 64 cache rows of a tile on the M side:
+//   S^T[tile rows, heads]  = C_tile (64 x 512, K-major)  *  Q~^T           (TMEM, fp32)
+//   O^T[latent, heads]    += C_tile^T (512 x 64, MN-major) * P^T           (TMEM, fp32)
+// so the latent dimension of O lives in TMEM lanes (4 blocks x 64 columns).  A tile
+// stays in shared memory from its score GEMM to its value GEMM, so every cache byte is
+// read once.  The ring holds 2.25 tiles: while the softmax works on tile t, the score
+// GEMM of tile t+1 runs and tile t+2 streams in; the MMA warp issues each tile's value
+// GEMM as soon as its probabilities are ready, which frees its ring slots.
 #include <math.h>
 
 #include <algorithm>
@@ -30,33 +33,40 @@
 namespace mla {
 namespace attend {
 
-constexpr int kTile = 128;                      // cache rows per tile (MMA M of the score GEMM)
+constexpr int kTile = 64;                       // cache rows per tile (MMA M of the score GEMM)
 constexpr int kRows = 64;                       // query rows per CTA = heads (MMA N)
-constexpr int kChunks = kLatent / 64;           // latent split in 128-byte swizzle columns
-constexpr int kChunkBytes = kTile * 64 * 2;     // 16 KB: 128 rows x 64 latent
+constexpr int kSlotQuarters = kLatent / 128;    // a tile is 4 ring slots of 128 latent values
+constexpr int kSlots = 9;                       // ring slots (2.25 tiles)
+constexpr int kAtomBytes = kTile * 128;         // 8 KB: 64 rows x 64 latent, 128-byte swizzle
+constexpr int kSlotBytes = 2 * kAtomBytes;      // 16 KB: 64 rows x 128 latent
+constexpr int kQtChunks = kLatent / 64;
 constexpr int kQtChunkBytes = kRows * 64 * 2;   // 8 KB: 64 heads x 64 latent
-constexpr int kPBytes = kTile * kRows * 2;      // 16 KB: P^T, 128 rows x 64 heads (bf16)
-constexpr int kThreads = 320;  // producer, MMA, 8 softmax warps
+constexpr int kPBytes = kTile * kRows * 2;      // 8 KB: P^T, 64 rows x 64 heads (bf16)
+constexpr int kThreads = 352;  // producer, score MMA, 8 softmax warps, value MMA
 constexpr int kSoftmaxWarps = 8;
 constexpr float kTau = 8.0f;  // lazy rescale: the running max is raised only when a score
                               // exceeds it by more than 2^8 (probabilities stay <= 256)
 
 constexpr int kOffC = 0;
-constexpr int kOffQt = kOffC + kChunks * kChunkBytes;
-constexpr int kOffP = kOffQt + kChunks * kQtChunkBytes;
-constexpr int kOffRed = kOffP + kPBytes;         // [4][64] floats
+constexpr int kOffQt = kOffC + kSlots * kSlotBytes;
+constexpr int kOffP = kOffQt + kQtChunks * kQtChunkBytes;
+constexpr int kOffRed = kOffP + 2 * kPBytes;     // [4][64] floats
 constexpr int kOffMUsed = kOffRed + 4 * 64 * 4;  // [64] floats
 constexpr int kOffAlpha = kOffMUsed + 64 * 4;    // [64] floats
 constexpr int kOffBar = kOffAlpha + 64 * 4;
 // barriers
-constexpr int kBarCFull = 0, kBarCEmpty = 8, kBarQFull = 16, kBarQEmpty = 17, kBarSFull = 18, kBarSEmpty = 20,
-              kBarPFull = 22, kBarPEmpty = 23, kBarOFull = 24, kBarOEmpty = 25, kNumBars = 26;
+constexpr int kBarCFull = 0, kBarCEmpty = kSlots, kBarQFull = 2 * kSlots, kBarQEmpty = kBarQFull + 1,
+              kBarSFull = kBarQEmpty + 1, kBarSEmpty = kBarSFull + 2, kBarPFull = kBarSEmpty + 2,
+              kBarPEmpty = kBarPFull + 2, kBarOFull = kBarPEmpty + 2, kBarOEmpty = kBarOFull + 1,
+              kNumBars = kBarOEmpty + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemUsed = kOffMisc + 16;
 constexpr int kSmemBytes = kSmemUsed + 1024;  // slack for 1024-byte alignment of the base
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kPageTokens == kTile, "a paged tile is exactly one page");
 
-// TMEM columns: two score buffers, then O^T as four 128-lane blocks of 64 columns.
+// TMEM columns: two score buffers (M = 64 accumulators: lanes 0-15 of each 32-lane
+// quadrant hold tile rows 16q..16q+15), then O^T as four 128-lane blocks of 64 columns.
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 0;
 constexpr uint32_t kTmemO = 256;
@@ -157,9 +167,9 @@ struct Shared {
   float *red, *m_used, *alpha;
   uint32_t *tmem_slot;
   volatile int *abort_flag;
-  __device__ uint8_t *chunk(int c) const { return base + kOffC + c * kChunkBytes; }
+  __device__ uint8_t *slot(int r) const { return base + kOffC + r * kSlotBytes; }
   __device__ uint8_t *qt(int c) const { return base + kOffQt + c * kQtChunkBytes; }
-  __device__ uint8_t *pbuf() const { return base + kOffP; }
+  __device__ uint8_t *pbuf(int i) const { return base + kOffP + i * kPBytes; }
 };
 
 __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, const Shared &sh, int32_t *status) {
@@ -167,10 +177,11 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, ok);
 }
 
+// Ring slot k (k = 4 * tile + quarter, counted over the CTA's tiles): position and use.
+__device__ __forceinline__ uint32_t ring_pos(uint32_t k) { return k % kSlots; }
+__device__ __forceinline__ uint32_t ring_use(uint32_t k) { return k / kSlots; }
+
 // ------------------------------------------------------------------ producer (warp 0)
-// Streams, per segment, q~ (64 heads x 512) once and then every tile's 8 latent chunks
-// into the 8-slot ring; slot c of tile t is refilled once the value GEMM of tile t-1 has
-// consumed chunk c.
 template <int kMode>
 __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUtensorMap *tm_cache,
                               const CUtensorMap *tm_qt, int iq, long long t0, long long t1, int lane) {
@@ -189,19 +200,19 @@ __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUt
       ok = mbar_wait(&bar[kBarQEmpty], (q_use & 1) ^ 1, sh.abort_flag, p.status);  // lane 0 only
     if (!ok) return;
     if (lane == 0) {
-      mbar_arrive_expect_tx(&bar[kBarQFull], kChunks * kQtChunkBytes);
+      mbar_arrive_expect_tx(&bar[kBarQFull], kQtChunks * kQtChunkBytes);
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c) tma_load_2d(sh.qt(c), tm_qt, &bar[kBarQFull], c * 64, qrow0);
+      for (int c = 0; c < kQtChunks; ++c) tma_load_2d(sh.qt(c), tm_qt, &bar[kBarQFull], c * 64, qrow0);
     }
     ++q_use;
     for (int t = sg.lo; t < sg.hi; ++t, ++tile_k) {
       if constexpr (kMode == kModeIndexed) {
-        // four tile rows per lane; rows past the list end are zero-filled
+        // two tile rows per lane; rows past the list end are zero-filled
         const int limit = query_limit(p, b, qi);
-        const uint16_t *src[4];
-        uint32_t nbytes[4];
+        const uint16_t *src[2];
+        uint32_t nbytes[2];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
+        for (int m = 0; m < 2; ++m) {
           const int k = t * kTile + lane + 32 * m;
           bool bad = false;
           long long row = 0;
@@ -210,44 +221,41 @@ __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUt
           src[m] = p.cache + row * kLatent;
           nbytes[m] = (k < p.K && !bad) ? 16u : 0u;
         }
-        for (int c = 0; c < kChunks; ++c) {
-          if (!wait_warp(&bar[kBarCEmpty + c], (tile_k & 1) ^ 1, sh, p.status)) return;
-          const uint32_t dst_c = smem_u32(sh.chunk(c));
+        for (int qq = 0; qq < kSlotQuarters; ++qq) {
+          const uint32_t k = tile_k * kSlotQuarters + qq;
+          const uint32_t rp = ring_pos(k);
+          if (!wait_warp(&bar[kBarCEmpty + rp], (ring_use(k) & 1) ^ 1, sh, p.status)) return;
+          const uint32_t dst_s = smem_u32(sh.slot(rp));
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
+          for (int m = 0; m < 2; ++m) {
             const int r = lane + 32 * m;
-            const uint32_t dst_r = dst_c + r * 128;
 #pragma unroll
-            for (int pc = 0; pc < 8; ++pc)
-              cp_async_16(dst_r + ((pc ^ (r & 7)) << 4), src[m] + c * 64 + pc * 8, nbytes[m]);
+            for (int at = 0; at < 2; ++at) {
+              const uint32_t dst_r = dst_s + at * kAtomBytes + r * 128;
+#pragma unroll
+              for (int pc = 0; pc < 8; ++pc)
+                cp_async_16(dst_r + ((pc ^ (r & 7)) << 4), src[m] + qq * 128 + at * 64 + pc * 8, nbytes[m]);
+            }
           }
-          cp_async_arrive_noinc(&bar[kBarCFull + c]);
+          cp_async_arrive_noinc(&bar[kBarCFull + rp]);
         }
       } else {
         const int j0 = t * kTile;
-        long long row[2] = {0, 0};
-        bool load[2];
-#pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-          const int jj = j0 + hb * 64;
-          load[hb] = jj < sg.rows;
-          if (load[hb]) {
-            if constexpr (kMode == kModePaged) {
-              bool bad = false;
-              row[hb] = paged_row(p.page_table, b, jj, p.max_pages, p.num_pages, bad);
-              if (bad) report_status(p.status, kStatusIndex);
-            } else {
-              row[hb] = dense_row(b, jj, p.Lmax);
-            }
-          }
+        long long row = 0;
+        if constexpr (kMode == kModePaged) {
+          bool bad = false;
+          row = paged_row(p.page_table, b, j0, p.max_pages, p.num_pages, bad);
+          if (bad) report_status(p.status, kStatusIndex);
+        } else {
+          row = dense_row(b, j0, p.Lmax);
         }
-        const uint32_t bytes = (load[0] ? 8192u : 0u) + (load[1] ? 8192u : 0u);
-        for (int c = 0; c < kChunks; ++c) {
-          if (!mbar_wait(&bar[kBarCEmpty + c], (tile_k & 1) ^ 1, sh.abort_flag, p.status)) return;
-          mbar_arrive_expect_tx(&bar[kBarCFull + c], bytes);
-#pragma unroll
-          for (int hb = 0; hb < 2; ++hb)
-            if (load[hb]) tma_load_2d(sh.chunk(c) + hb * 8192, tm_cache, &bar[kBarCFull + c], c * 64, (int)row[hb]);
+        for (int qq = 0; qq < kSlotQuarters; ++qq) {
+          const uint32_t k = tile_k * kSlotQuarters + qq;
+          const uint32_t rp = ring_pos(k);
+          if (!mbar_wait(&bar[kBarCEmpty + rp], (ring_use(k) & 1) ^ 1, sh.abort_flag, p.status)) return;
+          mbar_arrive_expect_tx(&bar[kBarCFull + rp], kSlotBytes);
+          tma_load_2d(sh.slot(rp), tm_cache, &bar[kBarCFull + rp], qq * 128, (int)row);
+          tma_load_2d(sh.slot(rp) + kAtomBytes, tm_cache, &bar[kBarCFull + rp], qq * 128 + 64, (int)row);
         }
       }
     }
@@ -255,93 +263,125 @@ __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUt
 }
 
 // ------------------------------------------------------------------ MMA issuer (warp 1)
-// Rows past the end of the sequence may hold any bits: zero them in the landed chunk so
+// Rows past the end of the sequence may hold any bits: zero them in the landed slot so
 // that a masked (zero) probability never meets a NaN or Inf in the value product.
 template <int kMode>
-__device__ __forceinline__ void prepare_chunk(uint32_t cbase, int n_valid, int lane) {
+__device__ __forceinline__ void prepare_slot(uint32_t sbase, int n_valid, int lane) {
   if (kMode != kModeIndexed && n_valid < kTile) {
-    for (int idx = lane; idx < (kTile - n_valid) * 8; idx += 32)
-      st_shared_v4(cbase + (n_valid + idx / 8) * 128 + (idx % 8) * 16, 0u, 0u, 0u, 0u);
+    const int n_zero = (kTile - n_valid) * 8;  // 16-byte units per atom
+    for (int idx = lane; idx < 2 * n_zero; idx += 32) {
+      const int at = idx / n_zero, u = idx % n_zero;
+      st_shared_v4(sbase + at * kAtomBytes + (n_valid + u / 8) * 128 + (u % 8) * 16, 0u, 0u, 0u, 0u);
+    }
     fence_proxy_async_smem();
   }
   if (kMode == kModeIndexed) fence_proxy_async_smem();  // rows written by 16-byte async copies
   __syncwarp();
 }
 
+// Two warps feed the tensor pipe with independent streams, each with plain blocking waits:
+// warp 1 issues the score GEMM of every tile, ring slot by ring slot as slots land, and
+// warp 10 issues the value GEMM of every tile as soon as its probabilities are ready (which
+// releases its ring slots).  MMAs of different threads are unordered, and the two streams
+// touch disjoint TMEM columns, so the pipe simply interleaves them.  Loop state and MMA
+// operands are warp-uniform; one elected lane issues.
 template <int kMode>
-__device__ void mma_role(const AttendParams &p, const Shared &sh, uint32_t tmem, long long t0, long long t1,
-                         int lane) {
+__device__ void score_mma_role(const AttendParams &p, const Shared &sh, uint32_t tmem, long long t0, long long t1,
+                               int lane) {
   uint64_t *bar = sh.bar;
-  constexpr uint32_t idesc_s = idesc_bf16_f32(128, kRows, false, false);
-  constexpr uint32_t idesc_o = idesc_bf16_f32(128, kRows, true, true);
-  uint32_t tile_k = 0, s_use = 0, p_use = 0, q_use = 0, o_use = 0;
-  const uint32_t c_base = smem_u32(sh.chunk(0));
+  constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kRows, false, false);
+  const uint32_t c_base = smem_u32(sh.slot(0));
   const uint32_t qt_base = smem_u32(sh.qt(0));
-  const uint32_t p_base = smem_u32(sh.pbuf());
+  uint32_t ns = 0, q_use = 0;
   SegIter it(t0, t1);
   Seg sg;
   while (it.next(p, kMode, sg)) {
     if (!wait_warp(&bar[kBarQFull], q_use & 1, sh, p.status)) return;
     ++q_use;
-    for (int t = sg.lo; t < sg.hi; ++t, ++tile_k) {
+    for (int t = sg.lo; t < sg.hi; ++t, ++ns) {
       const int n_valid = min(kTile, sg.rows - t * kTile);
-      // S^T[tile rows, heads] = C_tile * Q~^T, K = 512 latent in 8 chunks of 4 MMA steps
-      const uint32_t sb = s_use & 1;
-      if (!wait_warp(&bar[kBarSEmpty + sb], ((s_use >> 1) & 1) ^ 1, sh, p.status)) return;
-      tc_fence_after();
-      for (int c = 0; c < kChunks; ++c) {
-        if (!wait_warp(&bar[kBarCFull + c], tile_k & 1, sh, p.status)) return;
-        prepare_chunk<kMode>(c_base + c * kChunkBytes, n_valid, lane);
-        tc_fence_after();
-        if (lane == 0) {
+      if (!wait_warp(&bar[kBarSEmpty + (ns & 1)], ((ns >> 1) & 1) ^ 1, sh, p.status)) return;
+      const uint32_t d = tmem + kTmemS + (ns & 1) * kRows;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t a = sw128_desc(c_base + c * kChunkBytes + kk * 32, 16, 1024);
-            const uint64_t bdesc = sw128_desc(qt_base + c * kQtChunkBytes + kk * 32, 16, 1024);
-            umma_bf16(tmem + kTmemS + sb * kRows, a, bdesc, idesc_s, (c | kk) != 0);
+      for (uint32_t sq = 0; sq < kSlotQuarters; ++sq) {
+        // S^T[tile rows, heads] = C_tile * Q~^T; this slot holds K = 128 latent (8 steps)
+        const uint32_t k = ns * kSlotQuarters + sq;
+        if (!wait_warp(&bar[kBarCFull + ring_pos(k)], ring_use(k) & 1, sh, p.status)) return;
+        const uint32_t sbase = c_base + ring_pos(k) * kSlotBytes;
+        prepare_slot<kMode>(sbase, n_valid, lane);
+        tc_fence_after();
+        const uint64_t a0 = sw128_desc(sbase, 16, 1024);
+        const uint64_t b0 = sw128_desc(qt_base + 2 * sq * kQtChunkBytes, 16, 1024);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            // K step of 16 latent: 32 bytes inside a 128-byte swizzle row; the second four
+            // steps are in the slot's second atom (A) and the next q~ chunk (B)
+            const uint32_t ao = ((kk >> 2) * kAtomBytes + (kk & 3) * 32) >> 4;
+            const uint32_t bo = ((kk >> 2) * kQtChunkBytes + (kk & 3) * 32) >> 4;
+            umma_bf16(d, a0 + ao, b0 + bo, idesc_s, (sq != 0 || kk != 0) ? 1u : 0u);
           }
         }
         __syncwarp();
       }
-      if (lane == 0) {
-        umma_commit(&bar[kBarSFull + sb]);
+      if (elect_one()) {
+        umma_commit(&bar[kBarSFull + (ns & 1)]);
         if (t == sg.hi - 1) umma_commit(&bar[kBarQEmpty]);
-      }
-      ++s_use;
-      // O^T[latent, heads] += C_tile^T * P^T, four 128-lane latent blocks, K = 128 rows
-      if (!wait_warp(&bar[kBarPFull], p_use & 1, sh, p.status)) return;
-      ++p_use;
-      if (t == sg.lo && !wait_warp(&bar[kBarOEmpty], (o_use & 1) ^ 1, sh, p.status)) return;
-      tc_fence_after();
-      if (lane == 0) {
-#pragma unroll
-        for (int mb = 0; mb < 4; ++mb) {
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            // A = C_tile^T: latent (M) along the 128-byte rows, 64-wide atoms in the two
-            // chunks 2mb, 2mb+1 (LBO = chunk stride); cache rows (K) in 8-row groups.
-            const uint64_t a = sw128_desc(c_base + (2 * mb) * kChunkBytes + kk * 2048, kChunkBytes, 1024);
-            // B = P^T: heads (N) along the 128-byte rows, cache rows (K) in 8-row groups.
-            const uint64_t bdesc = sw128_desc(p_base + kk * 2048, 8192, 1024);
-            umma_bf16(tmem + kTmemO + mb * kRows, a, bdesc, idesc_o, (t > sg.lo || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(&bar[kBarCEmpty + 2 * mb]);
-          umma_commit(&bar[kBarCEmpty + 2 * mb + 1]);
-        }
-        umma_commit(&bar[kBarPEmpty]);
       }
       __syncwarp();
     }
-    if (lane == 0) umma_commit(&bar[kBarOFull]);
+  }
+}
+
+template <int kMode>
+__device__ void value_mma_role(const AttendParams &p, const Shared &sh, uint32_t tmem, long long t0, long long t1) {
+  uint64_t *bar = sh.bar;
+  constexpr uint32_t idesc_o = idesc_bf16_f32(128, kRows, true, true);
+  const uint32_t c_base = smem_u32(sh.slot(0));
+  const uint32_t p_base = smem_u32(sh.pbuf(0));
+  uint32_t no = 0, o_use = 0;
+  SegIter it(t0, t1);
+  Seg sg;
+  while (it.next(p, kMode, sg)) {
+    if (!wait_warp(&bar[kBarOEmpty], (o_use & 1) ^ 1, sh, p.status)) return;
+    for (int t = sg.lo; t < sg.hi; ++t, ++no) {
+      if (!wait_warp(&bar[kBarPFull + (no & 1)], (no >> 1) & 1, sh, p.status)) return;
+      tc_fence_after();
+      // O^T[latent, heads] += C_tile^T * P^T, four 128-lane latent blocks, K = 64 rows.
+      // A = C_tile^T: latent (M) along the 128-byte rows, 64-wide atoms LBO apart; cache
+      // rows (K) in 8-row groups.  B = P^T: heads (N) along the 128-byte rows, rows (K) in
+      // 8-row groups.  A K step of 16 rows advances both by 2 KB (128 in descriptor units).
+      const uint64_t b0 = sw128_desc(p_base + (no & 1) * kPBytes, kPBytes, 1024);
+      uint64_t a0[kSlotQuarters];
+      uint32_t rp[kSlotQuarters];
+#pragma unroll
+      for (int mb = 0; mb < kSlotQuarters; ++mb) {
+        rp[mb] = ring_pos(no * kSlotQuarters + mb);
+        a0[mb] = sw128_desc(c_base + rp[mb] * kSlotBytes, kAtomBytes, 1024);
+      }
+      const uint32_t acc0 = (t > sg.lo) ? 1u : 0u;
+      if (elect_one()) {
+#pragma unroll
+        for (int mb = 0; mb < kSlotQuarters; ++mb) {
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            umma_bf16(tmem + kTmemO + mb * kRows, a0[mb] + kk * 128, b0 + kk * 128, idesc_o, kk > 0 ? 1u : acc0);
+          umma_commit(&bar[kBarCEmpty + rp[mb]]);
+        }
+        umma_commit(&bar[kBarPEmpty + (no & 1)]);
+        if (t == sg.hi - 1) umma_commit(&bar[kBarOFull]);
+      }
+      __syncwarp();
+    }
     ++o_use;
   }
 }
 
 // ------------------------------------------------------------------ softmax + epilogue (warps 2-9)
-// Two warpgroups; warpgroup wg owns head columns [32 wg, 32 wg + 32) of S^T and O^T.  Thread
-// `row` of a warpgroup owns cache row `row` of the tile.  The running max per column lives
-// in shared memory (read with broadcast loads).  With 10 warps, three share an SM
-// sub-partition's register file, which caps a thread at 168 registers.
+// Two warpgroups; warpgroup wg owns head columns [32 wg, 32 wg + 32) of S^T and O^T.  Warp
+// quadrant wq holds tile rows 16 wq .. 16 wq + 15 (the M = 64 accumulator layout); thread t
+// owns rows 16 wq + t/4 and 16 wq + t/4 + 8 and the 8 head columns 8j + 2(t%4) + {0,1}.
+// The running max per column lives in shared memory and in registers.
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -355,16 +395,16 @@ __device__ void softmax_role(const AttendParams &p, const Shared &sh, uint32_t t
   const int wg = (warp - 2) >> 2;              // warpgroup: head columns [32 wg, 32 wg + 32)
   const int wq = warp & 3;                     // TMEM lane quadrant of this warp
   const int tid = ((warp - 2) & 3) * 32 + lane;  // 0..127 within the warpgroup
-  const int row = wq * 32 + lane;              // tile row (TMEM lane) owned by this thread
+  const int r0 = wq * 16 + (lane >> 2);        // tile rows r0 and r0 + 8 owned by this thread
+  const int cq = lane & 3;                     // column pair within each 8-column block
   const uint32_t bar_id = 1 + wg;
   const int col0 = wg * 32;
   const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
-  const uint32_t p_row = smem_u32(sh.pbuf()) + row * 128;
+  const uint32_t p_off = (uint32_t)r0 * 128 + cq * 4;
   float *red = sh.red;          // [4 quadrants][64 columns]
   float *m_used = sh.m_used;    // [64]
   float *alpha = sh.alpha;      // [64]
-  uint32_t s_use = 0, p_use = 0, o_use = 0;
-  const float *mu = m_used + col0;  // running max of this warpgroup's columns (log2 units)
+  uint32_t n = 0, o_use = 0;    // tiles seen by this CTA, segments finished
   if (tid < 32) m_used[col0 + tid] = -INFINITY;
   named_bar_sync(bar_id, 128);
   SegIter it(t0, t1);
@@ -373,38 +413,54 @@ __device__ void softmax_role(const AttendParams &p, const Shared &sh, uint32_t t
     const int qi = (kMode == kModeIndexed) ? sg.s % p.Q : iq;
     // positions of this CTA's query that are visible: dense/paged rows 0..L_b-Q+qi, or the list
     const int n_vis = (kMode == kModeIndexed) ? p.K : sg.rows - p.Q + qi + 1;
-    float l_part[32];
+    float l_part[8], m_reg[8];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) l_part[c] = 0.f;
-    for (int t = sg.lo; t < sg.hi; ++t) {
-      const uint32_t sb = s_use & 1;
-      mbar_wait(&bar[kBarSFull + sb], (s_use >> 1) & 1, sh.abort_flag, p.status);
+    for (int c = 0; c < 8; ++c) {
+      l_part[c] = 0.f;
+      m_reg[c] = -INFINITY;
+    }
+    for (int t = sg.lo; t < sg.hi; ++t, ++n) {
+      const uint32_t sb = n & 1;
+      mbar_wait(&bar[kBarSFull + sb], (n >> 1) & 1, sh.abort_flag, p.status);
       tc_fence_after();
-      const bool valid = (t * kTile + row) < n_vis;
-      float s2[32];
+      const bool v0 = (t * kTile + r0) < n_vis, v1 = (t * kTile + r0 + 8) < n_vis;
+      float s2[16];
       {
-        uint32_t r[32];
-        tmem_ld32(t_lane + kTmemS + sb * kRows + col0, r);
+        uint32_t r[16];
+        tmem_ld16x256_x4(t_lane + kTmemS + sb * kRows + col0, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) s2[c] = valid ? __uint_as_float(r[c]) * p.scale_log2 : -INFINITY;
+        for (int j = 0; j < 4; ++j) {
+          s2[4 * j + 0] = v0 ? __uint_as_float(r[4 * j + 0]) * p.scale_log2 : -INFINITY;
+          s2[4 * j + 1] = v0 ? __uint_as_float(r[4 * j + 1]) * p.scale_log2 : -INFINITY;
+          s2[4 * j + 2] = v1 ? __uint_as_float(r[4 * j + 2]) * p.scale_log2 : -INFINITY;
+          s2[4 * j + 3] = v1 ? __uint_as_float(r[4 * j + 3]) * p.scale_log2 : -INFINITY;
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[kBarSEmpty + sb]);
-      ++s_use;
+      // column h = 2j + e of this thread (j: 8-column block, e: pair member)
       bool flag = false;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) flag |= s2[c] > mu[c] + kTau;
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          flag |= fmaxf(s2[4 * j + e], s2[4 * j + 2 + e]) > m_reg[2 * j + e] + kTau;
       const bool any = named_bar_or(bar_id, 128, flag);
       if (*sh.abort_flag) return;
       if (any) {
         // new running max for this warpgroup's 32 columns
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float mx = warp_max_f32(s2[c]);
-          if (lane == c) red[wq * kRows + col0 + c] = mx;
-        }
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            float mx = fmaxf(s2[4 * j + e], s2[4 * j + 2 + e]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            if (lane < 4) red[wq * kRows + col0 + 8 * j + 2 * cq + e] = mx;
+          }
         named_bar_sync(bar_id, 128);
         if (tid < 32) {
           const int c = col0 + tid;
@@ -416,13 +472,21 @@ __device__ void softmax_role(const AttendParams &p, const Shared &sh, uint32_t t
         }
         named_bar_sync(bar_id, 128);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) l_part[c] *= alpha[col0 + c];
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = col0 + 8 * j + 2 * cq + e;
+            l_part[2 * j + e] *= alpha[c];
+            m_reg[2 * j + e] = m_used[c];
+          }
       }
-      // the P buffer is free and the previous value product has finished
-      mbar_wait(&bar[kBarPEmpty], (p_use & 1) ^ 1, sh.abort_flag, p.status);
-      tc_fence_after();
+      // this P buffer is free (the value product of tile n-2 has finished)
+      mbar_wait(&bar[kBarPEmpty + sb], ((n >> 1) & 1) ^ 1, sh.abort_flag, p.status);
       if (any && t > sg.lo) {
-        // running max moved: rescale this warpgroup's O^T columns in TMEM
+        // running max moved: once the value product of tile n-1 has finished, rescale this
+        // warpgroup's O^T columns in TMEM
+        mbar_wait(&bar[kBarPEmpty + (sb ^ 1)], ((n - 1) >> 1) & 1, sh.abort_flag, p.status);
+        tc_fence_after();
 #pragma unroll 1
         for (int mb = 0; mb < 4; ++mb) {
           uint32_t r[32];
@@ -436,36 +500,39 @@ __device__ void softmax_role(const AttendParams &p, const Shared &sh, uint32_t t
         tmem_st_wait();
       }
       // probabilities, rounded to bf16 for the value product; l sums the rounded values
+      const uint32_t pb = smem_u32(sh.pbuf(sb)) + p_off;
 #pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {
-        uint32_t w[4];
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t sw = (uint32_t)(((wg * 4 + j) ^ (r0 & 7)) << 4);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c0 = pc * 8 + 2 * e;
-          const float p0 = (s2[c0] == -INFINITY) ? 0.f : fast_exp2(s2[c0] - mu[c0]);
-          const float p1 = (s2[c0 + 1] == -INFINITY) ? 0.f : fast_exp2(s2[c0 + 1] - mu[c0 + 1]);
-          w[e] = pack_bf16x2(p0, p1);
-          l_part[c0] += bf16lo_to_f32(w[e]);
-          l_part[c0 + 1] += bf16hi_to_f32(w[e]);
+        for (int h = 0; h < 2; ++h) {  // h = 0: row r0, h = 1: row r0 + 8
+          const float x0 = s2[4 * j + 2 * h], x1 = s2[4 * j + 2 * h + 1];
+          const float p0 = (x0 == -INFINITY) ? 0.f : fast_exp2(x0 - m_reg[2 * j]);
+          const float p1 = (x1 == -INFINITY) ? 0.f : fast_exp2(x1 - m_reg[2 * j + 1]);
+          const uint32_t w = pack_bf16x2(p0, p1);
+          l_part[2 * j] += bf16lo_to_f32(w);
+          l_part[2 * j + 1] += bf16hi_to_f32(w);
+          st_shared_b32(pb + h * 8 * 128 + sw, w);
         }
-        st_shared_v4(p_row + (((wg * 4 + pc) ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[kBarPFull]);
-      ++p_use;
+      if (lane == 0) mbar_arrive(&bar[kBarPFull + sb]);
     }
     // ---- epilogue: l column sums, partial O, (m, l) -> workspace
     mbar_wait(&bar[kBarOFull], o_use & 1, sh.abort_flag, p.status);
     tc_fence_after();
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      float v = l_part[c];
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == c) red[wq * kRows + col0 + c] = v;
-    }
+      for (int e = 0; e < 2; ++e) {
+        float v = l_part[2 * j + e];
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        if (lane < 4) red[wq * kRows + col0 + 8 * j + 2 * cq + e] = v;
+      }
     named_bar_sync(bar_id, 128);
     if (*sh.abort_flag) return;
     const long long slot =
@@ -497,7 +564,9 @@ __device__ void softmax_role(const AttendParams &p, const Shared &sh, uint32_t t
 
 // ------------------------------------------------------------------ kernel
 template <int kMode>
-__global__ void __launch_bounds__(kThreads, 1)
+// Bounds for 384 threads: eleven warps put three on some SM sub-partitions, whose 16K
+// registers then cap a thread at 168 (the 352-thread bound alone would allow 184).
+__global__ void __launch_bounds__(384, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_qt,
                   const AttendParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -516,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int iq = blockIdx.x % p.group_size;
 
   if (threadIdx.x == 0) {
-    for (int c = 0; c < kChunks; ++c) {
+    for (int c = 0; c < kSlots; ++c) {
       mbar_init(&sh.bar[kBarCFull + c], kMode == kModeIndexed ? 32 : 1);
       mbar_init(&sh.bar[kBarCEmpty + c], 1);
     }
@@ -525,9 +594,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sh.bar[kBarSFull + i], 1);
       mbar_init(&sh.bar[kBarSEmpty + i], kSoftmaxWarps);
+      mbar_init(&sh.bar[kBarPFull + i], kSoftmaxWarps);
+      mbar_init(&sh.bar[kBarPEmpty + i], 1);
     }
-    mbar_init(&sh.bar[kBarPFull], kSoftmaxWarps);
-    mbar_init(&sh.bar[kBarPEmpty], 1);
     mbar_init(&sh.bar[kBarOFull], 1);
     mbar_init(&sh.bar[kBarOEmpty], kSoftmaxWarps);
     *sh.abort_flag = 0;
@@ -553,7 +622,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (kMode == kModeIndexed || lane == 0) producer_role<kMode>(p, sh, &tm_cache, &tm_qt, iq, t0, t1, lane);
   } else if (warp == 1) {
-    mma_role<kMode>(p, sh, tmem, t0, t1, lane);
+    score_mma_role<kMode>(p, sh, tmem, t0, t1, lane);
+  } else if (warp == 10) {
+    value_mma_role<kMode>(p, sh, tmem, t0, t1);
   } else {
     softmax_role<kMode>(p, sh, tmem, g, iq, t0, t1, warp, lane);
   }
