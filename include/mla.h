@@ -143,6 +143,40 @@ mla_status mla_attend_dense_noalloc(const uint16_t *q_tilde, const uint16_t *cac
                                     float *lse, int32_t *status, void *stream);
 
 /*
+ * Latent-cache bookkeeping around a speculative verify step.  Page "Module 08 -- Vision,
+ * MTP, and Hybrid Serving State" (jared-hpc.com, GLM-5.3-Flash Architecture Mastery,
+ * Lecture-08), section 3: the MLA latent cache is indexed by token position, so it is
+ * rolled back by truncating it to the accepted prefix, and the state after rollback must
+ * equal the state of a run that never generated the rejected tokens.
+ *
+ * mla_cache_append_*: write the Q latent rows of a verify window after each sequence's
+ * current length and advance the length:
+ *   rows     [B, Q, R] bf16     rows[b, i] goes to position seq_lens[b] + i
+ *   seq_lens [B] int32, in/out  seq_lens[b] += Q
+ *   dense:   cache [B, Lmax, R] bf16, position j of sequence b is cache[b, j]
+ *   paged:   pool [num_pages, page_size = 64, R] bf16, page_table [B, max_pages] int32;
+ *            position j is pool[page_table[b, j / 64], j % 64].  The caller maps the pages
+ *            first: every position written must land on an entry in [0, num_pages).
+ * mla_cache_truncate_*: keep the first keep[b] (0..Q) of the last Q rows of sequence b:
+ *   seq_lens[b] becomes seq_lens[b] - Q + keep[b] and the discarded rows are set to zero,
+ *   so a cache whose unused rows are zero ends identical to one that never held them.
+ *   Pages that become empty stay mapped; releasing them is the caller's business.
+ * A sequence whose positions would fall outside the cache (or on an unmapped or
+ * out-of-range page), or whose keep[b] is outside 0..Q, is left untouched and sets
+ * MLA_ERR_INDEX; the other sequences proceed.  Q >= 1, R = 512.
+ */
+mla_status mla_cache_append_dense(uint16_t *cache, int32_t *seq_lens, const uint16_t *rows, int B, int Q, int R,
+                                  int Lmax, int32_t *status, void *stream);
+mla_status mla_cache_append_paged(uint16_t *pool, const int32_t *page_table, int32_t *seq_lens, const uint16_t *rows,
+                                  int B, int Q, int R, int page_size, int max_pages, int num_pages, int32_t *status,
+                                  void *stream);
+mla_status mla_cache_truncate_dense(uint16_t *cache, int32_t *seq_lens, const int32_t *keep, int B, int Q, int R,
+                                    int Lmax, int32_t *status, void *stream);
+mla_status mla_cache_truncate_paged(uint16_t *pool, const int32_t *page_table, int32_t *seq_lens, const int32_t *keep,
+                                    int B, int Q, int R, int page_size, int max_pages, int num_pages, int32_t *status,
+                                    void *stream);
+
+/*
  * Bytes of workspace the mla_attend_* calls need for B sequences of Q queries on the
  * current device (split-L partial results and their max/sum terms).  0 on bad sizes.
  */

@@ -20,7 +20,8 @@ H, D, R, PAGE = 64, 256, 512, 64
 SCALE = 1.0 / 16.0
 
 EXPORTS = ("mla_status_string", "mla_last_error_string", "mla_absorb_q", "mla_attend_dense", "mla_attend_paged", "mla_attend_indexed",
-           "mla_up_proj", "mla_attend_workspace_bytes", "mla_debug_gather", "mla_attend_dense_noalloc")
+           "mla_up_proj", "mla_attend_workspace_bytes", "mla_debug_gather", "mla_attend_dense_noalloc",
+           "mla_cache_append_dense", "mla_cache_append_paged", "mla_cache_truncate_dense", "mla_cache_truncate_paged")
 
 
 class MLAError(RuntimeError):
@@ -55,8 +56,13 @@ def lib():
     L.mla_attend_workspace_bytes.restype = sz
     L.mla_debug_gather.argtypes = [i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp, vp, vp]
     L.mla_attend_dense_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp, vp, vp]
+    L.mla_cache_append_dense.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp]
+    L.mla_cache_truncate_dense.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp]
+    L.mla_cache_append_paged.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
+    L.mla_cache_truncate_paged.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
     for name in ("mla_absorb_q", "mla_up_proj", "mla_attend_dense", "mla_attend_paged", "mla_attend_indexed",
-                 "mla_debug_gather", "mla_attend_dense_noalloc"):
+                 "mla_debug_gather", "mla_attend_dense_noalloc", "mla_cache_append_dense", "mla_cache_append_paged",
+                 "mla_cache_truncate_dense", "mla_cache_truncate_paged"):
         getattr(L, name).restype = ctypes.c_int32
     _lib = L
     return L
@@ -200,6 +206,40 @@ def mla_debug_gather(mode, src, req, page_table=None, indices=None, B=None, Q=1,
         mode, _ptr(src), _ptr(page_table), _ptr(indices), B, Q, R, Lmax, max_pages, num_pages, K, _ptr(req), n,
         _ptr(out), _ptr(status), _stream(stream)))
     return out
+
+
+def mla_cache_append_dense(cache, seq_lens, rows, status=None, stream=None):
+    """Append rows [B, Q, R] bf16 at positions seq_lens[b] + i of cache [B, Lmax, R];
+    seq_lens [B] int32 advances by Q (in place)."""
+    _check_cuda(cache, seq_lens, rows, status)
+    B, Q = rows.shape[0], rows.shape[1]
+    _check("mla_cache_append_dense", lib().mla_cache_append_dense(
+        _ptr(cache), _ptr(seq_lens), _ptr(rows), B, Q, R, cache.shape[1], _ptr(status), _stream(stream)))
+
+
+def mla_cache_append_paged(pool, page_table, seq_lens, rows, status=None, stream=None):
+    """Append rows [B, Q, R] bf16 through page_table [B, max_pages] into pool [P, 64, R]."""
+    _check_cuda(pool, page_table, seq_lens, rows, status)
+    B, Q = rows.shape[0], rows.shape[1]
+    _check("mla_cache_append_paged", lib().mla_cache_append_paged(
+        _ptr(pool), _ptr(page_table), _ptr(seq_lens), _ptr(rows), B, Q, R, pool.shape[1], page_table.shape[1],
+        pool.shape[0], _ptr(status), _stream(stream)))
+
+
+def mla_cache_truncate_dense(cache, seq_lens, keep, q_len, status=None, stream=None):
+    """Keep the first keep[b] of the last q_len rows of each sequence; zero the rest."""
+    _check_cuda(cache, seq_lens, keep, status)
+    _check("mla_cache_truncate_dense", lib().mla_cache_truncate_dense(
+        _ptr(cache), _ptr(seq_lens), _ptr(keep), seq_lens.shape[0], q_len, R, cache.shape[1], _ptr(status),
+        _stream(stream)))
+
+
+def mla_cache_truncate_paged(pool, page_table, seq_lens, keep, q_len, status=None, stream=None):
+    """Paged counterpart of mla_cache_truncate_dense."""
+    _check_cuda(pool, page_table, seq_lens, keep, status)
+    _check("mla_cache_truncate_paged", lib().mla_cache_truncate_paged(
+        _ptr(pool), _ptr(page_table), _ptr(seq_lens), _ptr(keep), seq_lens.shape[0], q_len, R, pool.shape[1],
+        page_table.shape[1], pool.shape[0], _ptr(status), _stream(stream)))
 
 
 def mla_decode(q, w_uk, w_uv, cache, seq_lens=None, *, mode=MODE_DENSE, page_table=None, indices=None,

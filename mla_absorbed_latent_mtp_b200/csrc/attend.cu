@@ -606,6 +606,8 @@ __global__ void __launch_bounds__(384, 1)
     tmem_alloc(sh.tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  grid_dep_launch();
+  grid_dep_wait();  // inputs (q~, lengths, tables, cache) may come from the previous kernel
   // tile range of this CTA's group
   const long long T = warp_total_tiles(p, kMode, lane);
   const long long G = p.groups;
@@ -651,19 +653,19 @@ __global__ void __launch_bounds__(384, 1)
 
 // ------------------------------------------------------------------ combine
 // One block per (sequence b, query i) and pair of heads; thread t owns latent 4t..4t+3.
-// The partial of every CTA group that processed tiles of b is weighted by
-// 2^(m_g - M) (M the largest running max) and the weighted sums are normalised.
+// The partials of the CTA groups that processed tiles of b are merged online in chunks of
+// eight (all loads of a chunk in flight at once): with M the largest running max so far,
+// O = sum 2^(m_g - M) O_g and l = sum 2^(m_g - M) l_g, then O / l and lse = M + log2 l.
 constexpr int kCombineHeads = 2;
-constexpr int kMaxSlotsPerSeq = 1024;
+constexpr int kCombineChunk = 8;
 
 __global__ void __launch_bounds__(128) combine_kernel(const AttendParams p, int mode) {
+  grid_dep_launch();
+  grid_dep_wait();  // the partials come from the attend kernel just before
   const int v = blockIdx.x;  // b * Q + i
   const int b = v / p.Q, i = v % p.Q;
   const int s = (mode == kModeIndexed) ? v : b;
   __shared__ long long sh_info[3];
-  __shared__ float sh_w[kCombineHeads][kMaxSlotsPerSeq];
-  __shared__ float sh_l[kCombineHeads][kMaxSlotsPerSeq];
-  __shared__ float sh_norm[kCombineHeads][2];  // 1/den, lse
   const int tid = threadIdx.x;
   if (tid < 32) {
     const int ns = num_seqs(p, mode);
@@ -696,62 +698,69 @@ __global__ void __launch_bounds__(128) combine_kernel(const AttendParams p, int 
     g_first = ((ts + 1) * G - 1) / T;
     g_last = ((ts + nt) * G - 1) / T;
   }
-  const int nslot = (int)min(g_last - g_first + 1, (long long)kMaxSlotsPerSeq);
-  auto slot_of = [&](long long gg) -> long long {
-    return (mode == kModeIndexed) ? gg + s : (gg + s) * p.Q + i;
-  };
+  const int nslot = (int)(g_last - g_first + 1);
   const int h0 = blockIdx.y * kCombineHeads;
-  // weights: running maxima of the non-empty groups, then 2^(m - M) and the normaliser
-  for (int x = tid; x < kCombineHeads * nslot; x += 128) {
-    const int hh = x / nslot, k = x % nslot;
-    const long long gg = g_first + k;
-    float m = -INFINITY, l = 0.f;
-    if (group_start(gg, T, G) < group_start(gg + 1, T, G)) {
-      m = p.part_m[slot_of(gg) * kRows + h0 + hh];
-      l = p.part_l[slot_of(gg) * kRows + h0 + hh];
-    }
-    sh_w[hh][k] = m;
-    sh_l[hh][k] = l;
-  }
-  __syncthreads();
-  if (tid < kCombineHeads) {
-    const int hh = tid;
-    float M = -INFINITY;
-    for (int k = 0; k < nslot; ++k) M = fmaxf(M, sh_w[hh][k]);
-    float den = 0.f;
-    for (int k = 0; k < nslot; ++k) {
-      const float m = sh_w[hh][k];
-      const float w = (m == -INFINITY) ? 0.f : exp2f(m - M);
-      sh_w[hh][k] = w;
-      den += w * sh_l[hh][k];
-    }
-    const bool ok = (M != -INFINITY) && den > 0.f;
-    sh_norm[hh][0] = ok ? 1.f / den : 0.f;
-    sh_norm[hh][1] = ok ? (M + log2f(den)) * 0.69314718055994530942f : -INFINITY;
-  }
-  __syncthreads();
   const int lat = tid * 4;
+  float M[kCombineHeads], den[kCombineHeads];
+  float4 acc[kCombineHeads];
+#pragma unroll
+  for (int hh = 0; hh < kCombineHeads; ++hh) {
+    M[hh] = -INFINITY;
+    den[hh] = 0.f;
+    acc[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int k0 = 0; k0 < nslot; k0 += kCombineChunk) {
+    float mk[kCombineHeads][kCombineChunk], lk[kCombineHeads][kCombineChunk];
+    float4 ok[kCombineHeads][kCombineChunk];
+#pragma unroll
+    for (int j = 0; j < kCombineChunk; ++j) {
+      const long long gg = g_first + k0 + j;
+      const bool live = (k0 + j < nslot) && group_start(gg, T, G) < group_start(gg + 1, T, G);
+      const long long slot = (mode == kModeIndexed) ? gg + s : (gg + s) * p.Q + i;
+#pragma unroll
+      for (int hh = 0; hh < kCombineHeads; ++hh) {
+        const long long row = slot * kRows + h0 + hh;
+        mk[hh][j] = live ? p.part_m[row] : -INFINITY;
+        lk[hh][j] = live ? p.part_l[row] : 0.f;
+        ok[hh][j] = live ? *reinterpret_cast<const float4 *>(p.part_o + row * kLatent + lat)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < kCombineHeads; ++hh) {
+      float mx = M[hh];
+#pragma unroll
+      for (int j = 0; j < kCombineChunk; ++j) mx = fmaxf(mx, mk[hh][j]);
+      if (mx == -INFINITY) continue;
+      const float a = exp2f(M[hh] - mx);  // 0 when M was -inf
+      den[hh] *= a;
+      acc[hh].x *= a;
+      acc[hh].y *= a;
+      acc[hh].z *= a;
+      acc[hh].w *= a;
+#pragma unroll
+      for (int j = 0; j < kCombineChunk; ++j) {
+        const float w = exp2f(mk[hh][j] - mx);  // 0 for empty slots (m = -inf)
+        den[hh] += w * lk[hh][j];
+        acc[hh].x += w * ok[hh][j].x;
+        acc[hh].y += w * ok[hh][j].y;
+        acc[hh].z += w * ok[hh][j].z;
+        acc[hh].w += w * ok[hh][j].w;
+      }
+      M[hh] = mx;
+    }
+  }
 #pragma unroll
   for (int hh = 0; hh < kCombineHeads; ++hh) {
     const int h = h0 + hh;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int k = 0; k < nslot; ++k) {
-      const float w = sh_w[hh][k];
-      if (w != 0.f) {
-        const float4 o = *reinterpret_cast<const float4 *>(p.part_o + (slot_of(g_first + k) * kRows + h) * kLatent + lat);
-        acc.x += w * o.x;
-        acc.y += w * o.y;
-        acc.z += w * o.z;
-        acc.w += w * o.w;
-      }
-    }
-    const float inv = sh_norm[hh][0];
+    const bool good = (M[hh] != -INFINITY) && den[hh] > 0.f;
+    const float inv = good ? 1.f / den[hh] : 0.f;
     uint2 outv;
-    outv.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    outv.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    outv.x = pack_bf16x2(acc[hh].x * inv, acc[hh].y * inv);
+    outv.y = pack_bf16x2(acc[hh].z * inv, acc[hh].w * inv);
     *reinterpret_cast<uint2 *>(p.o_latent + ((long long)v * kRows + h) * kLatent + lat) = outv;
-    if (p.lse != nullptr && tid == 0) p.lse[(long long)v * kRows + h] = sh_norm[hh][1];
+    if (p.lse != nullptr && tid == 0)
+      p.lse[(long long)v * kRows + h] = good ? (M[hh] + log2f(den[hh])) * 0.69314718055994530942f : -INFINITY;
   }
 }
 
@@ -808,12 +817,11 @@ static cudaError_t launch_attend_mode(const CUtensorMap &tm_cache, const CUtenso
     configured_device = dev;
   }
   const int grid = p.groups * p.group_size;
-  attend::attend_kernel<kMode><<<grid, attend::kThreads, attend::kSmemBytes, stream>>>(tm_cache, tm_qt, p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_chained(attend::attend_kernel<kMode>, dim3(grid), dim3(attend::kThreads), attend::kSmemBytes,
+                                 stream, tm_cache, tm_qt, p);
   if (e != cudaSuccess) return e;
   dim3 cgrid(p.B * p.Q, kHeads / attend::kCombineHeads);
-  attend::combine_kernel<<<cgrid, 128, 0, stream>>>(p, kMode);
-  return cudaGetLastError();
+  return launch_chained(attend::combine_kernel, cgrid, dim3(128), 0, stream, p, (int)kMode);
 }
 
 cudaError_t launch_attend(int mode, const CUtensorMap &tm_cache, const CUtensorMap &tm_qt, const AttendParams &p,

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace mla {
 
 // Address modes of the attend kernel.
@@ -53,6 +55,27 @@ cudaError_t launch_proj(bool a_mn_major, const CUtensorMap &tm_w, const CUtensor
                         int M_total, int K_total, int n_tile, uint16_t *out, cudaStream_t stream);
 
 int device_sm_count();
+
+// Launch with programmatic stream serialization: the kernel may start while the previous
+// kernel in the stream is still running, once that kernel's CTAs have all signalled
+// (griddepcontrol.launch_dependents) or exited.  Every kernel of this library launched
+// this way executes griddepcontrol.wait before it reads anything an earlier kernel could
+// have written; before that it only initialises itself and reads weights.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                           Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 // Records e as the calling thread's last CUDA error; returns MLA_ERR_CUDA (MLA_OK for success).
 int32_t record_cuda_error(cudaError_t e);
 

@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int h = blockIdx.x, mb = blockIdx.y, nt = blockIdx.z;
+  grid_dep_launch();
   const int NT = p.n_tile;
   const int nk = p.K_total / kBK;
 
@@ -76,10 +77,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tensormap(&tm_w);
       prefetch_tensormap(&tm_x);
-      for (int kc = 0; kc < nk; ++kc) {
-        const int s = kc % kStages, use = kc / kStages;
-        if (!mbar_wait(&empty[s], (use & 1) ^ 1, abort_flag, nullptr)) break;
-        mbar_arrive_expect_tx(&full[s], kABytes + NT * kBK * 2);
+      auto load_a = [&](int kc, int s) {
         uint8_t *a_dst = a_stage0 + s * kABytes;
         if (kAMajorMN) {
           // W_UK[h][d][r]: box {64 r, 64 d}; two boxes cover the 128 r of this block
@@ -89,6 +87,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           // W_UV[h][d][r]: box {64 r, 128 d}
           tma_load_3d(a_dst, &tm_w, &full[s], kc * kBK, mb * kBM, h);
         }
+      };
+      // The weights never come from an earlier kernel: the first ring's worth streams in
+      // while the preceding kernel finishes; the token rows are read after it has.
+      const int pre = min(kStages, nk);
+      for (int kc = 0; kc < pre; ++kc) {
+        mbar_arrive_expect_tx(&full[kc], kABytes + NT * kBK * 2);
+        load_a(kc, kc);
+      }
+      grid_dep_wait();
+      for (int kc = 0; kc < pre; ++kc) tma_load_3d(b_stage0 + kc * b_bytes, &tm_x, &full[kc], kc * kBK, h, nt * NT);
+      for (int kc = pre; kc < nk; ++kc) {
+        const int s = kc % kStages, use = kc / kStages;
+        if (!mbar_wait(&empty[s], (use & 1) ^ 1, abort_flag, nullptr)) break;
+        mbar_arrive_expect_tx(&full[s], kABytes + NT * kBK * 2);
+        load_a(kc, s);
         tma_load_3d(b_stage0 + s * b_bytes, &tm_x, &full[s], kc * kBK, h, nt * NT);
       }
     }
@@ -100,23 +113,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&full[s], use & 1, abort_flag, nullptr));
       if (!ok) break;
       tc_fence_after();
-      if (lane == 0) {
-        const uint32_t a_base = smem_u32(a_stage0 + s * kABytes);
-        const uint32_t b_base = smem_u32(b_stage0 + s * b_bytes);
+      // MN-major A: 64-wide r atoms 8 KB apart (LBO), 8-row d groups 1 KB apart (SBO), K step
+      // = 2 KB; K-major A/B: 128-byte rows, 8-row groups 1 KB apart, K step = 32 bytes.
+      const uint64_t a0 = kAMajorMN ? sw128_desc(smem_u32(a_stage0 + s * kABytes), kABytes / 2, 1024)
+                                    : sw128_desc(smem_u32(a_stage0 + s * kABytes), 16, 1024);
+      const uint64_t b0 = sw128_desc(smem_u32(b_stage0 + s * b_bytes), 16, 1024);
+      if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          // MN-major A: 64-wide r atoms 8 KB apart (LBO), 8-row d groups 1 KB apart (SBO);
-          // K-major A/B: 128-byte rows, 8-row groups 1 KB apart, K step = 32 bytes.
-          const uint64_t a = kAMajorMN ? sw128_desc(a_base + kk * 2048, kABytes / 2, 1024)
-                                       : sw128_desc(a_base + kk * 32, 16, 1024);
-          const uint64_t b = sw128_desc(b_base + kk * 32, 16, 1024);
-          umma_bf16(tmem, a, b, idesc, (kc | kk) != 0);
-        }
+        for (int kk = 0; kk < kBK / 16; ++kk)
+          umma_bf16(tmem, a0 + (kAMajorMN ? kk * 128 : kk * 2), b0 + kk * 2, idesc, (kc | kk) != 0);
         umma_commit(&empty[s]);
       }
       __syncwarp();
     }
-    if (lane == 0) umma_commit(done);
+    if (elect_one()) umma_commit(done);
     __syncwarp();
   } else {
     const bool ok = mbar_wait(done, 0, abort_flag, nullptr);
@@ -163,8 +173,8 @@ static cudaError_t launch_proj_t(const CUtensorMap &tm_w, const CUtensorMap &tm_
     configured_device = dev;
   }
   dim3 grid(p.H, p.M_total / proj::kBM, (p.n + p.n_tile - 1) / p.n_tile);
-  proj::proj_kernel<kAMajorMN><<<grid, proj::kThreads, proj::smem_bytes(p.stages, p.n_tile), stream>>>(tm_w, tm_x, p);
-  return cudaGetLastError();
+  return launch_chained(proj::proj_kernel<kAMajorMN>, grid, dim3(proj::kThreads), proj::smem_bytes(p.stages, p.n_tile),
+                        stream, tm_w, tm_x, p);
 }
 
 cudaError_t launch_proj(bool a_mn_major, const CUtensorMap &tm_w, const CUtensorMap &tm_x, int n, int H,

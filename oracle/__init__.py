@@ -249,3 +249,51 @@ def up_project_all(o_bits: np.ndarray, w_uv_bits: np.ndarray) -> np.ndarray:
     for h in range(o.shape[1]):
         out[:, h, :] = o[:, h, :] @ u[h].T
     return out
+
+
+# ----------------------------------------------------------------------------- speculative-decoding cache bookkeeping
+# "Module 08 -- Vision, MTP, and Hybrid Serving State" (jared-hpc.com, GLM-5.3-Flash
+# Architecture Mastery, Lecture-08), section 3: the MLA latent cache is indexed by token
+# position, so after a verify step it is rolled back by truncating it to the accepted
+# prefix, and the state after rollback must equal the state of a run that never produced
+# the rejected tokens.  The MTP page (dimsnsums.com, GLM-5.3-Flash MTP): a verify step
+# appends the q_len = 1 + 5 rows it scores.  These are plain array assignments on bits.
+
+def _slot(mode: str, b: int, j: int, page_table):
+    """(array index) of logical position j of sequence b: cache[b, j] or pool[page, j % 64]."""
+    if mode == "paged":
+        page = int(page_table[b, j // PAGE_TOKENS])
+        if page < 0:
+            raise ValueError("position maps to an unused page-table slot")
+        return (page, j % PAGE_TOKENS)
+    return (b, j)
+
+
+def cache_append(mode: str, store: np.ndarray, seq_lens: np.ndarray, rows: np.ndarray, page_table=None):
+    """Append rows[b, i] (bits, [B, q_len, R]) at positions seq_lens[b] + i.
+
+    Returns new (store, seq_lens); the inputs are not modified."""
+    store = np.array(store, copy=True)
+    lens = np.array(seq_lens, dtype=np.int64, copy=True)
+    B, q_len = rows.shape[0], rows.shape[1]
+    for b in range(B):
+        for i in range(q_len):
+            store[_slot(mode, b, int(lens[b]) + i, page_table)] = rows[b, i]
+        lens[b] += q_len
+    return store, lens.astype(np.int32)
+
+
+def cache_truncate(mode: str, store: np.ndarray, seq_lens: np.ndarray, keep: np.ndarray, q_len: int,
+                   page_table=None):
+    """Roll back a verify window: sequence b keeps the first keep[b] of its last q_len rows.
+
+    The new length is seq_lens[b] - q_len + keep[b]; the discarded rows are zeroed, so a
+    store whose unused rows are zero ends up identical to one that never held them."""
+    store = np.array(store, copy=True)
+    lens = np.array(seq_lens, dtype=np.int64, copy=True)
+    for b in range(len(lens)):
+        new_len = int(lens[b]) - q_len + int(keep[b])
+        for j in range(new_len, int(lens[b])):
+            store[_slot(mode, b, j, page_table)] = 0
+        lens[b] = new_len
+    return store, lens.astype(np.int32)
