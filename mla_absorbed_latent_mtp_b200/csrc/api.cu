@@ -138,6 +138,8 @@ static mla_status attend_common(int mode, const uint16_t *q_tilde, const uint16_
   p.part_o = reinterpret_cast<float *>(workspace);
   p.part_m = p.part_o + slots * kHeads * kLatent;
   p.part_l = p.part_m + slots * kHeads;
+  p.seq_ts = reinterpret_cast<long long *>(p.part_l + slots * kHeads);
+  p.seq_nt = reinterpret_cast<int32_t *>(p.seq_ts + (size_t)B * Q);
   p.o_latent = o_latent;
   p.lse = lse;
   p.status = status;

@@ -100,6 +100,28 @@ __device__ long long warp_total_tiles(const AttendParams &p, int mode, int lane)
 
 __device__ __forceinline__ long long group_start(long long g, long long T, long long G) { return g * T / G; }
 
+// Position of every sequence in the tile list (first tile, tile count), for the combine
+// (computed by one warp with an exclusive scan in steps of 32 sequences).
+__device__ void warp_write_seq_prefix(const AttendParams &p, int mode, int lane) {
+  const int ns = num_seqs(p, mode);
+  long long base = 0;
+  for (int s0 = 0; s0 < ns; s0 += 32) {
+    const int s = s0 + lane;
+    const int nt = s < ns ? seq_tiles(p, mode, s) : 0;
+    long long x = nt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (s < ns) {
+      p.seq_ts[s] = base + x - nt;
+      p.seq_nt[s] = nt;
+    }
+    base += __shfl_sync(0xffffffffu, x, 31);
+  }
+}
+
 struct Seg {
   int s;      // sequence in the tile list
   int lo, hi; // tile range within the sequence
@@ -144,15 +166,19 @@ __device__ __forceinline__ long long paged_row(const int32_t *table, int b, int 
   return (long long)page * kPageTokens + (j % kPageTokens);
 }
 
-// Indexed: list position k of query i of sequence b; valid entries lie in [0, limit].
-__device__ __forceinline__ long long indexed_row(const int32_t *indices, int b, int i, int k, int Q, int K,
-                                                 int Lmax, int limit, bool &bad) {
-  const int j = indices[((long long)b * Q + i) * K + k];
+// Indexed: row of list entry j of sequence b; valid entries lie in [0, limit] and below Lmax.
+__device__ __forceinline__ long long indexed_row_of(int b, int j, int Lmax, int limit, bool &bad) {
   if (j < 0 || j > limit || j >= Lmax) {
     bad = true;
     return 0;
   }
   return (long long)b * Lmax + j;
+}
+
+// Indexed: list position k of query i of sequence b.
+__device__ __forceinline__ long long indexed_row(const int32_t *indices, int b, int i, int k, int Q, int K,
+                                                 int Lmax, int limit, bool &bad) {
+  return indexed_row_of(b, indices[((long long)b * Q + i) * K + k], Lmax, limit, bad);
 }
 
 __device__ __forceinline__ int query_limit(const AttendParams &p, int b, int i) {
@@ -205,10 +231,29 @@ __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUt
       for (int c = 0; c < kQtChunks; ++c) tma_load_2d(sh.qt(c), tm_qt, &bar[kBarQFull], c * 64, qrow0);
     }
     ++q_use;
+    // indexed: the list entries of the next tile are read while this tile's rows are
+    // copied (two rows per lane), so the index load latency is off the copy path
+    const int32_t *list = p.indices + ((long long)b * p.Q + qi) * p.K;
+    int nxt[2] = {0, 0};
+    if constexpr (kMode == kModeIndexed) {
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int k = sg.lo * kTile + lane + 32 * m;
+        if (k < p.K) nxt[m] = list[k];
+      }
+    }
     for (int t = sg.lo; t < sg.hi; ++t, ++tile_k) {
       if constexpr (kMode == kModeIndexed) {
         // two tile rows per lane; rows past the list end are zero-filled
         const int limit = query_limit(p, b, qi);
+        const int cur[2] = {nxt[0], nxt[1]};
+        if (t + 1 < sg.hi) {
+#pragma unroll
+          for (int m = 0; m < 2; ++m) {
+            const int k = (t + 1) * kTile + lane + 32 * m;
+            if (k < p.K) nxt[m] = list[k];
+          }
+        }
         const uint16_t *src[2];
         uint32_t nbytes[2];
 #pragma unroll
@@ -216,7 +261,7 @@ __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUt
           const int k = t * kTile + lane + 32 * m;
           bool bad = false;
           long long row = 0;
-          if (k < p.K) row = indexed_row(p.indices, b, qi, k, p.Q, p.K, p.Lmax, limit, bad);
+          if (k < p.K) row = indexed_row_of(b, cur[m], p.Lmax, limit, bad);
           if (bad) report_status(p.status, kStatusIndex);
           src[m] = p.cache + row * kLatent;
           nbytes[m] = (k < p.K && !bad) ? 16u : 0u;
@@ -611,6 +656,7 @@ __global__ void __launch_bounds__(384, 1)
   // tile range of this CTA's group
   const long long T = warp_total_tiles(p, kMode, lane);
   const long long G = p.groups;
+  if (blockIdx.x == 0 && warp == 0) warp_write_seq_prefix(p, kMode, lane);
   const long long t0 = group_start(g, T, G), t1 = group_start(g + 1, T, G);
   tc_fence_before();
   __syncthreads();
@@ -652,47 +698,31 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 // ------------------------------------------------------------------ combine
-// One block per (sequence b, query i) and pair of heads; thread t owns latent 4t..4t+3.
-// The partials of the CTA groups that processed tiles of b are merged online in chunks of
-// eight (all loads of a chunk in flight at once): with M the largest running max so far,
-// O = sum 2^(m_g - M) O_g and l = sum 2^(m_g - M) l_g, then O / l and lse = M + log2 l.
+// One block per (query row v = b * Q + i) and pair of heads; thread t owns latent 4t..4t+3
+// of both heads.  The partials of the CTA groups that processed tiles of the row's
+// sequence are merged online in chunks of eight, all loads of a chunk in flight at once:
+// with M the largest running max so far, O = sum 2^(m_g - M) O_g and l = sum 2^(m_g - M) l_g,
+// then O / l and lse = M + log2 l.  The sequence's place in the tile list comes from the
+// table the attend kernel wrote.
 constexpr int kCombineHeads = 2;
 constexpr int kCombineChunk = 8;
 
-__global__ void __launch_bounds__(128) combine_kernel(const AttendParams p, int mode) {
+__global__ void __launch_bounds__(128, 4) combine_kernel(const AttendParams p, int mode) {
   grid_dep_launch();
   grid_dep_wait();  // the partials come from the attend kernel just before
   const int v = blockIdx.x;  // b * Q + i
   const int b = v / p.Q, i = v % p.Q;
   const int s = (mode == kModeIndexed) ? v : b;
-  __shared__ long long sh_info[3];
   const int tid = threadIdx.x;
-  if (tid < 32) {
-    const int ns = num_seqs(p, mode);
-    long long before = 0, total = 0;
-    for (int x = tid; x < ns; x += 32) {
-      const int nt = seq_tiles(p, mode, x);
-      total += nt;
-      if (x < s) before += nt;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      before += __shfl_xor_sync(0xffffffffu, before, o);
-      total += __shfl_xor_sync(0xffffffffu, total, o);
-    }
-    if (tid == 0) {
-      sh_info[0] = before;
-      sh_info[1] = seq_tiles(p, mode, s);
-      sh_info[2] = total;
-      if (blockIdx.y == 0 && i == 0 && mode != kModeIndexed && p.seq_lens != nullptr) {
-        const int L = p.seq_lens[b];
-        const int cap = (mode == kModePaged) ? p.max_pages * kPageTokens : p.Lmax;
-        if (L < 0 || L > cap) report_status(p.status, kStatusIndex);
-      }
-    }
+  const int ns = num_seqs(p, mode);
+  const long long T = p.seq_ts[ns - 1] + p.seq_nt[ns - 1], G = p.groups;
+  const long long ts = p.seq_ts[s];
+  const int nt = p.seq_nt[s];
+  if (tid == 0 && blockIdx.y == 0 && i == 0 && mode != kModeIndexed && p.seq_lens != nullptr) {
+    const int L = p.seq_lens[b];
+    const int cap = (mode == kModePaged) ? p.max_pages * kPageTokens : p.Lmax;
+    if (L < 0 || L > cap) report_status(p.status, kStatusIndex);
   }
-  __syncthreads();
-  const long long ts = sh_info[0], nt = sh_info[1], T = sh_info[2], G = p.groups;
   long long g_first = 0, g_last = -1;
   if (nt > 0) {
     g_first = ((ts + 1) * G - 1) / T;
@@ -801,7 +831,10 @@ size_t attend_slots(int B, int Q, int sms) {
 
 size_t attend_workspace_bytes_for(int B, int Q, int sms) {
   const size_t slots = attend_slots(B, Q, sms);
-  return slots * kHeads * kLatent * sizeof(float) + 2 * slots * kHeads * sizeof(float);
+  // partial O, m and l per slot, then per sequence of the tile list (at most B*Q of them)
+  // its first tile (int64) and tile count (int32)
+  return slots * kHeads * kLatent * sizeof(float) + 2 * slots * kHeads * sizeof(float) +
+         (size_t)B * (size_t)Q * (sizeof(long long) + sizeof(int32_t));
 }
 
 template <int kMode>

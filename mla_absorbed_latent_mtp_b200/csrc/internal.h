@@ -32,6 +32,8 @@ struct AttendParams {
   float *part_o;              // [slots, H, R] unnormalised partial outputs
   float *part_m;              // [slots, H] running max (log2 units)
   float *part_l;              // [slots, H] running sum
+  long long *seq_ts;          // [num_seqs] tiles of the list before sequence s (written by CTA 0)
+  int32_t *seq_nt;            // [num_seqs] tiles of sequence s
   uint16_t *o_latent;         // [B, Q, H, R] result
   float *lse;                 // [B, Q, H] or null
   int32_t *status;
