@@ -106,7 +106,10 @@ mla_status mla_attend_paged(const uint16_t *q_tilde, const uint16_t *pool, const
  * such as the DSA indexer's): query i of sequence b attends exactly to the rows
  * cache[b, indices[b, i, k]] for k < K.
  *   indices  [B, Q, K] int32   positions, each in [0, L_b - Q + i] (causally visible);
- *                              order does not matter, a repeated entry counts twice.
+ *                              order does not matter, a repeated entry counts twice;
+ *                              an entry of -1 is unused and contributes nothing (lists of a
+ *                              fixed width K that hold fewer positions, as the k-pool index
+ *                              producer below emits).
  *   seq_lens [B] int32 or NULL  as for mla_attend_dense (used to validate indices)
  * An out-of-range entry sets MLA_ERR_INDEX.  K >= 1.
  */
@@ -177,6 +180,33 @@ mla_status mla_cache_truncate_paged(uint16_t *pool, const int32_t *page_table, i
                                     void *stream);
 
 /*
+ * k-pool index producer for mla_attend_indexed.  Page "GLM-5.3-Flash engine (c/glm53.c)"
+ * (colibri docs), Architecture notes, DSA with k-pooling: keys are grouped into pools of
+ * `pool` consecutive positions, a pool's key is a per-channel softmax mixture of its
+ * members, only complete and causally visible pools are selectable, the incomplete tail is
+ * appended when asked for, and ties go to the lower index.  The pages give no indexer
+ * projections: here the key of a position is its cached latent c_j and the indexer query
+ * is a given vector w[b, i] of width R.
+ *
+ * mla_kpool_keys: pooled[b, p, d] = sum_j softmax_j(c[b, p*pool + j, d]) * c[b, p*pool + j, d]
+ *   for every complete pool of sequence b (p < seq_lens[b] / pool); other rows untouched.
+ *   cache [B, Lmax, R] bf16, seq_lens [B] int32 or NULL (all Lmax), pooled [B, Lmax / pool, R]
+ *   fp32 (caller-owned; may be reused across calls while the cache only grows).
+ * mla_kpool_select: for query i of sequence b at position t = seq_lens[b] - Q + i, writes
+ *   indices[b, i, 0 .. W) =
+ *     the positions of the topk / pool best pools among those ending at or before t
+ *     (score = w[b, i] . pooled[b, p] in fp32; ties to the lower pool), in ascending order,
+ *     then -1 up to topk; with_tail != 0 appends the positions of the incomplete pool up
+ *     to t, then -1 up to W = topk + pool - 1 (W = topk without the tail).
+ *   w_query [B, Q, R] bf16.  topk a positive multiple of pool, topk / pool <= 1024,
+ *   Lmax / pool <= 51200.  The list feeds mla_attend_indexed with K = W (-1 entries unused).
+ */
+mla_status mla_kpool_keys(const uint16_t *cache, const int32_t *seq_lens, int B, int R, int Lmax, int pool,
+                          float *pooled, void *stream);
+mla_status mla_kpool_select(const float *pooled, const uint16_t *w_query, const int32_t *seq_lens, int B, int Q, int R,
+                            int Lmax, int pool, int topk, int with_tail, int32_t *indices, int W, void *stream);
+
+/*
  * Bytes of workspace the mla_attend_* calls need for B sequences of Q queries on the
  * current device (split-L partial results and their max/sum terms).  0 on bad sizes.
  */
@@ -196,6 +226,15 @@ size_t mla_attend_workspace_bytes(int B, int Q, int H, int R);
 mla_status mla_debug_gather(int mode, const uint16_t *src, const int32_t *page_table, const int32_t *indices,
                             int B, int Q, int R, int Lmax, int max_pages, int num_pages, int K,
                             const int32_t *req, int n_req, uint16_t *out, int32_t *status, void *stream);
+
+/*
+ * Test aid for failure detection: runs the bounded mbarrier wait that every pipeline role
+ * of the attend kernel uses, on a barrier that nothing ever completes, with a limit of
+ * `limit_cycles` SM cycles (1 .. 2e9).  The wait gives up, writes MLA_ERR_TIMEOUT to
+ * *status (a device int32, required) if it is still MLA_OK, and the kernel returns: the
+ * context stays usable.  No counterpart on the pages.
+ */
+mla_status mla_debug_wait_timeout(long long limit_cycles, int32_t *status, void *stream);
 
 #ifdef __cplusplus
 }

@@ -21,7 +21,8 @@ SCALE = 1.0 / 16.0
 
 EXPORTS = ("mla_status_string", "mla_last_error_string", "mla_absorb_q", "mla_attend_dense", "mla_attend_paged", "mla_attend_indexed",
            "mla_up_proj", "mla_attend_workspace_bytes", "mla_debug_gather", "mla_attend_dense_noalloc",
-           "mla_cache_append_dense", "mla_cache_append_paged", "mla_cache_truncate_dense", "mla_cache_truncate_paged")
+           "mla_cache_append_dense", "mla_cache_append_paged", "mla_cache_truncate_dense", "mla_cache_truncate_paged",
+           "mla_debug_wait_timeout", "mla_kpool_keys", "mla_kpool_select")
 
 
 class MLAError(RuntimeError):
@@ -60,6 +61,12 @@ def lib():
     L.mla_cache_truncate_dense.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp]
     L.mla_cache_append_paged.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
     L.mla_cache_truncate_paged.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
+    L.mla_kpool_keys.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp]
+    L.mla_kpool_keys.restype = ctypes.c_int32
+    L.mla_kpool_select.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
+    L.mla_kpool_select.restype = ctypes.c_int32
+    L.mla_debug_wait_timeout.argtypes = [ctypes.c_longlong, vp, vp]
+    L.mla_debug_wait_timeout.restype = ctypes.c_int32
     for name in ("mla_absorb_q", "mla_up_proj", "mla_attend_dense", "mla_attend_paged", "mla_attend_indexed",
                  "mla_debug_gather", "mla_attend_dense_noalloc", "mla_cache_append_dense", "mla_cache_append_paged",
                  "mla_cache_truncate_dense", "mla_cache_truncate_paged"):
@@ -240,6 +247,38 @@ def mla_cache_truncate_paged(pool, page_table, seq_lens, keep, q_len, status=Non
     _check("mla_cache_truncate_paged", lib().mla_cache_truncate_paged(
         _ptr(pool), _ptr(page_table), _ptr(seq_lens), _ptr(keep), seq_lens.shape[0], q_len, R, pool.shape[1],
         page_table.shape[1], pool.shape[0], _ptr(status), _stream(stream)))
+
+
+def mla_debug_wait_timeout(limit_cycles, status, stream=None):
+    """Run the pipeline's bounded wait on a barrier nothing completes (test aid)."""
+    _check_cuda(status)
+    _check("mla_debug_wait_timeout", lib().mla_debug_wait_timeout(int(limit_cycles), _ptr(status), _stream(stream)))
+
+
+def mla_kpool_keys(cache, pool, seq_lens=None, pooled=None, stream=None):
+    """Pooled keys [B, Lmax // pool, R] fp32 of every complete pool of cache [B, Lmax, R]."""
+    import torch
+    _check_cuda(cache, seq_lens, pooled)
+    B, Lmax = cache.shape[0], cache.shape[1]
+    if pooled is None:
+        pooled = torch.zeros(B, Lmax // pool, R, dtype=torch.float32, device=cache.device)
+    _check("mla_kpool_keys", lib().mla_kpool_keys(_ptr(cache), _ptr(seq_lens), B, R, Lmax, pool, _ptr(pooled),
+                                                  _stream(stream)))
+    return pooled
+
+
+def mla_kpool_select(pooled, w_query, pool, topk, seq_lens=None, with_tail=True, Lmax=None, stream=None):
+    """Index lists [B, Q, topk (+ pool - 1)] int32 for w_query [B, Q, R] bf16."""
+    import torch
+    _check_cuda(pooled, w_query, seq_lens)
+    B, Q = w_query.shape[0], w_query.shape[1]
+    Lmax = pooled.shape[1] * pool if Lmax is None else Lmax
+    W = topk + (pool - 1 if with_tail else 0)
+    out = torch.empty(B, Q, W, dtype=torch.int32, device=w_query.device)
+    _check("mla_kpool_select", lib().mla_kpool_select(
+        _ptr(pooled), _ptr(w_query), _ptr(seq_lens), B, Q, R, Lmax, pool, topk, 1 if with_tail else 0, _ptr(out), W,
+        _stream(stream)))
+    return out
 
 
 def mla_decode(q, w_uk, w_uv, cache, seq_lens=None, *, mode=MODE_DENSE, page_table=None, indices=None,

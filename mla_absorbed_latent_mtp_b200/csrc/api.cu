@@ -254,4 +254,9 @@ mla_status mla_debug_gather(int mode, const uint16_t *src, const int32_t *page_t
                                                   K, req, n_req, out, status, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+mla_status mla_debug_wait_timeout(long long limit_cycles, int32_t *status, void *stream) {
+  if (status == nullptr || limit_cycles < 1 || limit_cycles > 2000000000LL) return MLA_ERR_ARG;
+  return mla::cuda_status(mla::launch_wait_timeout(limit_cycles, status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -181,6 +181,9 @@ __device__ __forceinline__ long long indexed_row(const int32_t *indices, int b, 
   return indexed_row_of(b, indices[((long long)b * Q + i) * K + k], Lmax, limit, bad);
 }
 
+// An index-list entry of -1 is unused (fixed-width lists shorter than their width).
+constexpr int kUnusedEntry = -1;
+
 __device__ __forceinline__ int query_limit(const AttendParams &p, int b, int i) {
   const int L = p.seq_lens ? p.seq_lens[b] : p.Lmax;
   return L - p.Q + i;  // position of query i; it sees rows 0..limit
@@ -261,10 +264,11 @@ __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUt
           const int k = t * kTile + lane + 32 * m;
           bool bad = false;
           long long row = 0;
-          if (k < p.K) row = indexed_row_of(b, cur[m], p.Lmax, limit, bad);
+          const bool used = k < p.K && cur[m] != kUnusedEntry;
+          if (used) row = indexed_row_of(b, cur[m], p.Lmax, limit, bad);
           if (bad) report_status(p.status, kStatusIndex);
           src[m] = p.cache + row * kLatent;
-          nbytes[m] = (k < p.K && !bad) ? 16u : 0u;
+          nbytes[m] = (used && !bad) ? 16u : 0u;
         }
         for (int qq = 0; qq < kSlotQuarters; ++qq) {
           const uint32_t k = tile_k * kSlotQuarters + qq;
@@ -464,11 +468,38 @@ __device__ void softmax_role(const AttendParams &p, const Shared &sh, uint32_t t
       l_part[c] = 0.f;
       m_reg[c] = -INFINITY;
     }
+    // indexed: the list entries of this thread's two rows of the next tile are read ahead
+    // (a -1 entry is unused and its row is masked)
+    const int32_t *list = (kMode == kModeIndexed)
+                              ? p.indices + ((long long)(sg.s / p.Q) * p.Q + (sg.s % p.Q)) * p.K
+                              : nullptr;
+    int ent_next[2] = {0, 0};
+    if constexpr (kMode == kModeIndexed) {
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int k = sg.lo * kTile + r0 + 8 * h2;
+        if (k < p.K) ent_next[h2] = list[k];
+      }
+    }
     for (int t = sg.lo; t < sg.hi; ++t, ++n) {
       const uint32_t sb = n & 1;
+      int ent[2] = {ent_next[0], ent_next[1]};
+      if constexpr (kMode == kModeIndexed) {
+        if (t + 1 < sg.hi) {
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int k = (t + 1) * kTile + r0 + 8 * h2;
+            if (k < p.K) ent_next[h2] = list[k];
+          }
+        }
+      }
       mbar_wait(&bar[kBarSFull + sb], (n >> 1) & 1, sh.abort_flag, p.status);
       tc_fence_after();
-      const bool v0 = (t * kTile + r0) < n_vis, v1 = (t * kTile + r0 + 8) < n_vis;
+      bool v0 = (t * kTile + r0) < n_vis, v1 = (t * kTile + r0 + 8) < n_vis;
+      if constexpr (kMode == kModeIndexed) {
+        v0 = v0 && ent[0] != kUnusedEntry;
+        v1 = v1 && ent[1] != kUnusedEntry;
+      }
       float s2[16];
       {
         uint32_t r[16];
@@ -819,7 +850,27 @@ __global__ void debug_gather_kernel(int mode, const uint16_t *src, const int32_t
   for (int x = threadIdx.x; x < R; x += blockDim.x) out[(long long)r * R + x] = bad ? 0 : src[row * R + x];
 }
 
+// ------------------------------------------------------------------ bounded-wait check
+// The bounded mbarrier wait of every pipeline role, on a barrier that nothing completes:
+// it must give up after about `limit` SM cycles, record MLA_ERR_TIMEOUT and return.
+__global__ void wait_timeout_kernel(long long limit, int32_t *status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  mbar_wait(&bar, 0, &abort_flag, status, limit);
+}
+
 }  // namespace attend
+
+cudaError_t launch_wait_timeout(long long limit_cycles, int32_t *status, cudaStream_t stream) {
+  attend::wait_timeout_kernel<<<1, 32, 0, stream>>>(limit_cycles, status);
+  return cudaGetLastError();
+}
 
 // ------------------------------------------------------------------ host launchers
 size_t attend_slots(int B, int Q, int sms) {

@@ -57,6 +57,7 @@ cudaError_t launch_proj(bool a_mn_major, const CUtensorMap &tm_w, const CUtensor
                         int M_total, int K_total, int n_tile, uint16_t *out, cudaStream_t stream);
 
 int device_sm_count();
+cudaError_t launch_wait_timeout(long long limit_cycles, int32_t *status, cudaStream_t stream);
 
 // Launch with programmatic stream serialization: the kernel may start while the previous
 // kernel in the stream is still running, once that kernel's CTAs have all signalled

@@ -78,14 +78,14 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // A complete phase is seen by one non-blocking probe; otherwise the thread sleeps in the
 // barrier (up to 1 ms per probe) instead of spinning.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                          int32_t *status) {
+                                          int32_t *status, long long limit_cycles = kWaitLimitCycles) {
   const uint32_t a = smem_u32(bar);
   if (mbar_test_wait(a, parity)) return true;  // cheap when the phase is already complete
   const long long t0 = clock64();
   while (true) {
     if (*abort_flag) return false;
     if (mbar_try_wait_sleep(a, parity, 1000000u)) return true;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit_cycles) {
       *abort_flag = 1;
       report_status(status, kStatusTimeout);
       return false;

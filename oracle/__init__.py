@@ -146,7 +146,8 @@ def up_project(o: np.ndarray, u_v: np.ndarray) -> np.ndarray:
 
 def _visible(wl, b: int, i: int) -> np.ndarray:
     if wl.mode == "indexed":
-        return np.asarray(wl.indices[b, i], dtype=np.int64)
+        lst = np.asarray(wl.indices[b, i], dtype=np.int64)
+        return lst[lst != -1]  # -1 marks an unused entry of a fixed-width list
     return visible_positions(int(wl.seq_lens[b]), wl.Q, i)
 
 
@@ -297,3 +298,39 @@ def cache_truncate(mode: str, store: np.ndarray, seq_lens: np.ndarray, keep: np.
             store[_slot(mode, b, j, page_table)] = 0
         lens[b] = new_len
     return store, lens.astype(np.int32)
+
+
+# ----------------------------------------------------------------------------- k-pool index producer
+# "GLM-5.3-Flash engine (c/glm53.c)" (colibri docs, raw.githubusercontent.com/JustVugg/colibri),
+# section "Architecture notes", DSA with k-pooling: keys are grouped into pools of
+# `pool` consecutive positions; the pooled key is a per-channel softmax mixture of the
+# members (not their average); a pool is selectable only if it is complete and causally
+# visible; the incomplete tail is appended when asked for (a row topk + pool - 1 wide);
+# ties go to the lower index.  The pages give no indexer projections, so the key of a
+# position is its cached latent and the indexer query is an input vector w.
+
+def kpool_pooled_keys(rows_bits: np.ndarray, pool: int) -> np.ndarray:
+    """Pooled key of every complete pool of consecutive rows ([n, R] bits -> [n // pool, R]):
+    per channel d, sum_j softmax_j(x_jd) * x_jd over the pool's members j."""
+    x = widen(rows_bits)
+    n_pools = x.shape[0] // pool
+    x = x[: n_pools * pool].reshape(n_pools, pool, x.shape[1])
+    e = np.exp(x - x.max(axis=1, keepdims=True))
+    return (e * x).sum(axis=1) / e.sum(axis=1)
+
+
+def kpool_select(pooled: np.ndarray, w: np.ndarray, pos: int, pool: int, topk: int, with_tail: bool) -> np.ndarray:
+    """Index list of the query at position `pos`: the topk // pool best complete pools that end
+    at or before pos (score = pooled . w, ties to the lower pool), their positions in
+    ascending order, then -1 up to topk; with_tail appends the positions of the incomplete
+    pool up to pos, then -1 up to topk + pool - 1."""
+    n_sel = max(pos + 1, 0) // pool
+    scores = pooled[:n_sel] @ np.asarray(w, dtype=np.float64)
+    order = sorted(range(n_sel), key=lambda p: (-scores[p], p))
+    chosen = sorted(order[: topk // pool])
+    out = [p * pool + j for p in chosen for j in range(pool)]
+    out += [-1] * (topk - len(out))
+    if with_tail:
+        tail = list(range(n_sel * pool, pos + 1))
+        out += tail + [-1] * (pool - 1 - len(tail))
+    return np.asarray(out, dtype=np.int32)

@@ -98,6 +98,21 @@ def test_debug_gather_rejects_host_errors(lib):
     assert f(0, GOOD, None, None, 1, 1, 512, 8, 0, 0, 0, GOOD, 0, GOOD, None, None) == m.MLA_OK
 
 
+def test_cache_bookkeeping_and_timeout_aid_reject_host_errors(lib):
+    p = ctypes.c_void_p(16)
+    # null store / lengths / rows, non-positive sizes, unsupported latent width
+    assert lib.mla_cache_append_dense(None, p, p, 1, 1, 512, 8, None, None) == m.MLA_ERR_ARG
+    assert lib.mla_cache_append_dense(p, p, p, 0, 1, 512, 8, None, None) == m.MLA_ERR_ARG
+    assert lib.mla_cache_append_dense(p, p, p, 1, 0, 512, 8, None, None) == m.MLA_ERR_ARG
+    assert lib.mla_cache_append_dense(p, p, p, 1, 1, 256, 8, None, None) == m.MLA_ERR_UNSUPPORTED
+    assert lib.mla_cache_truncate_dense(p, p, None, 1, 1, 512, 8, None, None) == m.MLA_ERR_ARG
+    assert lib.mla_cache_append_paged(p, None, p, p, 1, 1, 512, 64, 4, 4, None, None) == m.MLA_ERR_ARG
+    assert lib.mla_cache_append_paged(p, p, p, p, 1, 1, 512, 32, 4, 4, None, None) == m.MLA_ERR_UNSUPPORTED
+    assert lib.mla_cache_truncate_paged(p, p, p, p, 1, 1, 512, 64, 0, 4, None, None) == m.MLA_ERR_ARG
+    assert lib.mla_debug_wait_timeout(1000, None, None) == m.MLA_ERR_ARG
+    assert lib.mla_debug_wait_timeout(0, p, None) == m.MLA_ERR_ARG
+
+
 def test_product_path_does_not_touch_oracle():
     """The binding and kernels never import the oracle (test infrastructure only)."""
     pkg = os.path.join(ROOT, "mla_absorbed_latent_mtp_b200")
