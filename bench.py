@@ -38,8 +38,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one attend launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
 # ncu capture summarised in profiles/, keyed by the hash of the kernel source it was taken on.
 TRAFFIC = {
-    ("dense_decode", "4b7a6c6cf977435e"): 278_524_416,
-    ("mtp_verify", "4b7a6c6cf977435e"): 557_148_160,
+    ("dense_decode", "846e235ef9181498"): 277_537_536,
+    ("mtp_verify", "846e235ef9181498"): 556_857_600,
 }
 
 
