@@ -1,7 +1,8 @@
 // sm100.cuh -- thin inline-PTX wrappers for the Blackwell (sm_100a) features the
 // kernels use: mbarriers with bounded waits, TMA tensor loads (no multicast),
-// Ampere-style 16-byte async copies, and the tcgen05 tensor-core family
-// (TMEM allocation, MMA with shared-memory descriptors, commit, TMEM loads/stores).
+// 16-byte async copies, the tcgen05 tensor-core family (TMEM allocation, MMA with
+// shared-memory descriptors issued from an elected lane, commit, TMEM loads/stores),
+// named barriers, and programmatic dependent launch (griddepcontrol).
 #pragma once
 
 #include <cuda.h>
@@ -42,15 +43,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                    smem_u32(bar)),
                "r"(bytes)
                : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
 }
 // Non-blocking probe of a phase (try_wait may suspend the thread for a while first).
 __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
@@ -126,11 +118,6 @@ __device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t nthreads, boo
       : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
       : "memory");
   return out != 0;
-}
-__device__ __forceinline__ float warp_max_f32(float v) {
-  float r;
-  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
-  return r;
 }
 
 // ------------------------------------------------------------------ TMA (tensor) loads
