@@ -286,3 +286,39 @@ def test_full_path_small_against_expanded_oracle(mode, Q, lens, K):
     got = bf16_to_f64(out)
     for (b, i), r in ref.items():
         _assert_gate(got[b, i], r["out"], f"{mode} b={b} i={i}")
+
+
+# ----------------------------------------------------------------------------- split edge cases
+
+@pytest.mark.parametrize("mode", ["dense", "paged"])
+def test_zero_length_sequence_among_others(mode):
+    """A sequence with no rows has no tiles: its output is 0 and its lse -inf, and the
+    other sequences' splits are unaffected."""
+    lens = [300, 0, 65, 1]
+    wl = tiny_workload(mode, len(lens), 1, lens, H=64, D=256, R=512, seed=41)
+    qt = synthetic_qtilde(wl.B, 1, seed=42)
+    o, lse, st = _run_attend(wl, qt)
+    assert st == 0
+    _check_latent(wl, qt, o, lse)
+    assert not bool(torch.isfinite(lse[1]).any()) and not bool(o[1].any())
+
+
+def test_one_long_sequence_split_over_every_group():
+    """A single sequence spread over all CTA groups: about one partial per SM to merge."""
+    L = 100_000
+    wl = tiny_workload("dense", 1, 1, [L], H=64, D=256, R=512, seed=43)
+    qt = synthetic_qtilde(1, 1, seed=44)
+    o, lse, st = _run_attend(wl, qt)
+    assert st == 0
+    _check_latent(wl, qt, o, lse)
+
+
+def test_many_short_sequences():
+    """More sequences than SMs, each a single partial tile."""
+    lens = [1 + (7 * b) % 64 for b in range(300)]
+    wl = tiny_workload("dense", len(lens), 1, lens, H=64, D=256, R=512, seed=45)
+    qt = synthetic_qtilde(wl.B, 1, seed=46)
+    o, lse, st = _run_attend(wl, qt)
+    assert st == 0
+    pairs = [(b, 0) for b in range(0, len(lens), 37)]
+    _check_latent(wl, qt, o, lse, pairs=pairs)
