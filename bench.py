@@ -287,13 +287,9 @@ def main(argv=None):
     args = parse_args(argv)
     world, rank, local = dist_env()
     if args.impl == "reference":
-        if world > 1:
-            import torch.distributed as dist
-            dist.init_process_group("gloo")
-            run_reference(args, args.config)
-            dist.destroy_process_group()
-        else:
-            run_reference(args, args.config)
+        # under torchrun rank 0 alone runs the oracle; the other ranks exit without work
+        # (no process group: nothing is exchanged)
+        run_reference(args, args.config)
         return
 
     import numpy as np
