@@ -27,9 +27,10 @@ namespace mla {
 namespace kpool {
 
 constexpr int kThreads = 128;        // pool kernel: 4 channels per thread
-constexpr int kSelectThreads = 256;  // select kernel: 8 warps
+constexpr int kSelectThreads = 1024;  // select kernel: 32 warps
 constexpr int kMaxChosen = 1024;     // topk / pool bound (shared-memory list)
 constexpr int kChunkRows = 16;       // pool members per step of the pooling
+constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t v) { return __uint_as_float((uint32_t)v << 16); }
 
@@ -72,13 +73,14 @@ __global__ void __launch_bounds__(kThreads) pool_kernel(const uint16_t *cache, c
         float cm = m[c];
 #pragma unroll
         for (int r = 0; r < kChunkRows; ++r) cm = fmaxf(cm, x[r][c]);
-        const float a = expf(m[c] - cm);  // 0 on the first chunk
+        const float cm2 = cm * kLog2e;
+        const float a = exp2f(m[c] * kLog2e - cm2);  // 0 on the first chunk
         s[c] *= a;
         ws[c] *= a;
 #pragma unroll
         for (int r = 0; r < kChunkRows; ++r) {
           if (r < nr) {
-            const float e = expf(x[r][c] - cm);
+            const float e = exp2f(fmaf(x[r][c], kLog2e, -cm2));
             s[c] += e;
             ws[c] += e * x[r][c];
           }
@@ -117,17 +119,29 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const float *poo
     const uint16_t *wq = w_query + (long long)v * kLatent + lane * 16;
 #pragma unroll
     for (int c = 0; c < 16; ++c) w[c] = bf16_to_f32(wq[c]);
-    for (int p = warp; p < n_sel; p += kSelectThreads / 32) {
-      const float4 *row = reinterpret_cast<const float4 *>(pooled + ((long long)b * max_pools + p) * kLatent + lane * 16);
-      float acc = 0.f;
+    constexpr int kWarps = kSelectThreads / 32;
+    for (int p0 = warp; p0 < n_sel; p0 += 2 * kWarps) {  // two pools per pass, loads in flight together
+      float acc[2] = {0.f, 0.f};
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        const float4 x = row[c4];
-        acc += x.x * w[4 * c4] + x.y * w[4 * c4 + 1] + x.z * w[4 * c4 + 2] + x.w * w[4 * c4 + 3];
+      for (int u = 0; u < 2; ++u) {
+        const int p = p0 + u * kWarps;
+        if (p < n_sel) {
+          const float4 *row =
+              reinterpret_cast<const float4 *>(pooled + ((long long)b * max_pools + p) * kLatent + lane * 16);
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const float4 x = row[c4];
+            acc[u] += x.x * w[4 * c4] + x.y * w[4 * c4 + 1] + x.z * w[4 * c4 + 2] + x.w * w[4 * c4 + 3];
+          }
+        }
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) sh_score[p] = acc;
+      for (int u = 0; u < 2; ++u) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
+        const int p = p0 + u * kWarps;
+        if (lane == 0 && p < n_sel) sh_score[p] = acc[u];
+      }
     }
   }
   __syncthreads();
