@@ -53,6 +53,9 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--next-rows", action="store_true",
+                    help="time the cache bookkeeping and k-pool producer entry points instead")
+    ap.add_argument("--kpool-seqs", type=int, default=4, help="sequences of 131,072 rows for --next-rows")
     return ap.parse_args(argv)
 
 
@@ -283,9 +286,69 @@ def _truncated(wl, rows):
 
 # ----------------------------------------------------------------------------- our arm
 
+def run_next_rows(args):
+    """Event timing (median) of the latent-cache bookkeeping and the k-pool index producer:
+    append / truncate on the verify shape (B=16, q_len=6, 32,768-row prefix), pooled keys and
+    selection on --kpool-seqs sequences of 131,072 rows (pools of 64, topk 2,048 + tail)."""
+    import numpy as np
+    import torch
+
+    import mla_absorbed_latent_mtp_b200 as m
+    import synth
+    from mla_absorbed_latent_mtp_b200 import _build
+
+    _build.build()
+    torch.cuda.set_device(0)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+
+    def dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+    B, Q, L0 = 16, 6, 32768
+    cache = torch.zeros(B, L0 + 64, 512, dtype=torch.bfloat16, device="cuda")
+    lens = torch.full((B,), L0, dtype=torch.int32, device="cuda")
+    rows = dev(synth.normal_bf16((B, Q, 512), 1, synth.STREAM_Q))
+    keep = torch.full((B,), 3, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ta, tt = [], []
+    for k in range(args.warmup + args.steps):
+        lens.fill_(L0)
+        ev[0].record(); m.mla_cache_append_dense(cache, lens, rows, st); ev[1].record()
+        m.mla_cache_truncate_dense(cache, lens, keep, Q, st); ev[2].record()
+        torch.cuda.synchronize()
+        if k >= args.warmup:
+            ta.append(ev[0].elapsed_time(ev[1])); tt.append(ev[1].elapsed_time(ev[2]))
+    B2, L2, pool, topk = args.kpool_seqs, 131072, 64, 2048
+    c2 = dev(synth.normal_bf16((B2, L2, 512), 2, synth.STREAM_CACHE))
+    l2 = torch.full((B2,), L2, dtype=torch.int32, device="cuda")
+    wq = dev(synth.normal_bf16((B2, 1, 512), 3, synth.STREAM_Q))
+    pooled = torch.zeros(B2, L2 // pool, 512, dtype=torch.float32, device="cuda")
+    tk, ts = [], []
+    for k in range(args.warmup + args.steps):
+        ev[0].record(); m.mla_kpool_keys(c2, pool, l2, pooled); ev[1].record()
+        m.mla_kpool_select(pooled, wq, pool, topk, l2, True, Lmax=L2); ev[2].record()
+        torch.cuda.synchronize()
+        if k >= args.warmup:
+            tk.append(ev[0].elapsed_time(ev[1])); ts.append(ev[1].elapsed_time(ev[2]))
+    assert int(st.item()) == 0, m.status_string(int(st.item()))
+    med = lambda x: float(np.median(x)) * 1e3  # noqa: E731
+    print(json.dumps({
+        "next_rows": True, "unit": "us", "steps": args.steps, "warmup": args.warmup,
+        "cache_append_dense_us": med(ta), "cache_truncate_dense_us": med(tt),
+        "cache_shape": {"B": B, "q_len": Q, "prefix": L0, "keep": 3},
+        "kpool_keys_us": med(tk), "kpool_keys_gbs": B2 * L2 * 1024 / (med(tk) * 1e-6) / 1e9,
+        "kpool_select_us": med(ts),
+        "kpool_shape": {"B": B2, "rows": L2, "pool": pool, "topk": topk, "tail": True, "queries": B2},
+    }))
+
+
 def main(argv=None):
     args = parse_args(argv)
     world, rank, local = dist_env()
+    if args.next_rows:
+        if rank == 0:
+            run_next_rows(args)
+        return
     if args.impl == "reference":
         # under torchrun rank 0 alone runs the oracle; the other ranks exit without work
         # (no process group: nothing is exchanged)
