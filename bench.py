@@ -38,8 +38,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one attend launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
 # ncu capture summarised in profiles/, keyed by the hash of the kernel source it was taken on.
 TRAFFIC = {
-    ("dense_decode", "b535bd9d98201748"): 277_674_240,
-    ("mtp_verify", "b535bd9d98201748"): 556_614_912,
+    ("dense_decode", "14d6ff085e50bf20"): 277_809_920,
+    ("mtp_verify", "14d6ff085e50bf20"): 556_551_680,
 }
 
 

@@ -731,12 +731,13 @@ __global__ void __launch_bounds__(384, 1)
 // ------------------------------------------------------------------ combine
 // One block per (query row v = b * Q + i) and pair of heads; thread t owns latent 4t..4t+3
 // of both heads.  The partials of the CTA groups that processed tiles of the row's
-// sequence are merged online in chunks of eight, all loads of a chunk in flight at once:
+// sequence are merged online in chunks of six (every partial of the benchmark shapes in
+// one chunk), all loads of a chunk in flight at once:
 // with M the largest running max so far, O = sum 2^(m_g - M) O_g and l = sum 2^(m_g - M) l_g,
 // then O / l and lse = M + log2 l.  The sequence's place in the tile list comes from the
 // table the attend kernel wrote.
 constexpr int kCombineHeads = 2;
-constexpr int kCombineChunk = 8;
+constexpr int kCombineChunk = 6;
 
 __global__ void __launch_bounds__(128, 4) combine_kernel(const AttendParams p, int mode) {
   grid_dep_launch();
