@@ -746,21 +746,34 @@ __global__ void __launch_bounds__(128, 4) combine_kernel(const AttendParams p, i
   const int b = v / p.Q, i = v % p.Q;
   const int s = (mode == kModeIndexed) ? v : b;
   const int tid = threadIdx.x;
-  const int ns = num_seqs(p, mode);
-  const long long T = p.seq_ts[ns - 1] + p.seq_nt[ns - 1], G = p.groups;
-  const long long ts = p.seq_ts[s];
-  const int nt = p.seq_nt[s];
-  if (tid == 0 && blockIdx.y == 0 && i == 0 && mode != kModeIndexed && p.seq_lens != nullptr) {
-    const int L = p.seq_lens[b];
-    const int cap = (mode == kModePaged) ? p.max_pages * kPageTokens : p.Lmax;
-    if (L < 0 || L > cap) report_status(p.status, kStatusIndex);
+  const long long G = p.groups;
+  // The sequence's group range is block-uniform and costs 64-bit divisions: one thread
+  // computes it.  A group is empty only when there are fewer tiles than groups.
+  __shared__ long long sh_T, sh_g_first;
+  __shared__ int sh_nslot;
+  if (tid == 0) {
+    const int ns = num_seqs(p, mode);
+    const long long T = p.seq_ts[ns - 1] + p.seq_nt[ns - 1];
+    const long long ts = p.seq_ts[s];
+    const int nt = p.seq_nt[s];
+    long long g_first = 0, g_last = -1;
+    if (nt > 0) {
+      g_first = ((ts + 1) * G - 1) / T;
+      g_last = ((ts + nt) * G - 1) / T;
+    }
+    sh_T = T;
+    sh_g_first = g_first;
+    sh_nslot = (int)(g_last - g_first + 1);
+    if (blockIdx.y == 0 && i == 0 && mode != kModeIndexed && p.seq_lens != nullptr) {
+      const int L = p.seq_lens[b];
+      const int cap = (mode == kModePaged) ? p.max_pages * kPageTokens : p.Lmax;
+      if (L < 0 || L > cap) report_status(p.status, kStatusIndex);
+    }
   }
-  long long g_first = 0, g_last = -1;
-  if (nt > 0) {
-    g_first = ((ts + 1) * G - 1) / T;
-    g_last = ((ts + nt) * G - 1) / T;
-  }
-  const int nslot = (int)(g_last - g_first + 1);
+  __syncthreads();
+  const long long T = sh_T, g_first = sh_g_first;
+  const int nslot = sh_nslot;
+  const bool all_live = T >= G;
   const int h0 = blockIdx.y * kCombineHeads;
   const int lat = tid * 4;
   float M[kCombineHeads], den[kCombineHeads];
@@ -777,7 +790,7 @@ __global__ void __launch_bounds__(128, 4) combine_kernel(const AttendParams p, i
 #pragma unroll
     for (int j = 0; j < kCombineChunk; ++j) {
       const long long gg = g_first + k0 + j;
-      const bool live = (k0 + j < nslot) && group_start(gg, T, G) < group_start(gg + 1, T, G);
+      const bool live = (k0 + j < nslot) && (all_live || group_start(gg, T, G) < group_start(gg + 1, T, G));
       const long long slot = (mode == kModeIndexed) ? gg + s : (gg + s) * p.Q + i;
 #pragma unroll
       for (int hh = 0; hh < kCombineHeads; ++hh) {
