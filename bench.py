@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "latent-cache attention: effective HBM GB/s & TFLOP/s vs B200 roofline, 1 GPU"
 UNIT = "GB/s"
+L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic of one attend launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
@@ -105,54 +106,94 @@ def kernel_source_hash():
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
+    """SM clock and clock-event reasons sampled while the timed loop runs.
+
+    NVML is polled about once a millisecond from a thread (a timed region of a few tens
+    of milliseconds still gets samples); without NVML, ``nvidia-smi -lms 50`` is read
+    instead.  Only samples taken inside the timed window count: with none there, the
+    summary says "unsampled" rather than reporting idle clocks."""
     QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NVML_REASONS = ((0x4, "sw_power_cap"), (0x8, "hw_slowdown"), (0x20, "sw_thermal_slowdown"),
+                    (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"))
 
-    def __init__(self, index):
+    def __init__(self, index, pci_bus_id=None):
         self.index = index
+        self.pci_bus_id = pci_bus_id
         self.proc = None
-        self.lines = []
+        self.rows = []  # (wall time, sm MHz, max sm MHz, [reason names])
+        self.source = None
+        self._stop = threading.Event()
+        self.thread = None
 
     def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            if self.pci_bus_id:
+                h = pynvml.nvmlDeviceGetHandleByPciBusId(self.pci_bus_id)
+            else:
+                h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.source = "nvml 1 ms"
+            self.thread = threading.Thread(target=self._poll_nvml, args=(pynvml, h, max_mhz), daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            pass
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
                                           "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.source = "nvidia-smi 50 ms"
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
             self.thread.start()
         except OSError:
             self.proc = None
 
-    def _read(self):
+    def _poll_nvml(self, pynvml, h, max_mhz):
+        while not self._stop.is_set():
+            try:
+                mhz = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                bits = int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))
+            except Exception:
+                return
+            self.rows.append((time.time(), mhz, max_mhz, [n for b, n in self.NVML_REASONS if bits & b]))
+            time.sleep(0.001)
+
+    def _read_smi(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.proc.stdout:
-            self.lines.append((time.time(), line.strip()))
+            parts = [x.strip() for x in line.strip().split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                self.rows.append((time.time(), float(parts[2]), float(parts[3]),
+                                  [names[k] for k, v in enumerate(parts[6:10]) if v.lower() == "active"]))
+            except ValueError:
+                continue
 
     def stop(self):
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
     def summary(self, t0, t1):
-        rows = []
-        for ts, line in self.lines:
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 10:
-                continue
-            try:
-                rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
-            except ValueError:
-                continue
-        window = [r for r in rows if t0 <= r[0] <= t1] or rows
+        window = [r for r in self.rows if t0 <= r[0] <= t1]
         if not window:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for r in window for k, v in enumerate(r[3]) if v.lower() == "active"})
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0,
+                    "source": self.source}
+        reasons = sorted({n for r in window for n in r[3]})
         return {"sm_mhz": statistics.median(r[1] for r in window), "sm_max_mhz": max(r[2] for r in window),
-                "reasons": reasons, "samples": len(window)}
+                "sm_mhz_min": min(r[1] for r in window), "reasons": reasons, "samples": len(window),
+                "source": self.source}
 
 
 # ----------------------------------------------------------------------------- distributed helpers
@@ -391,6 +432,16 @@ def main(argv=None):
     host_lens = torch.from_numpy(wl.seq_lens).pin_memory()
     table = torch.from_numpy(wl.page_table).to(device) if wl.mode == "paged" else None
     idx = torch.from_numpy(wl.indices).to(device) if wl.mode == "indexed" else None
+    # the rows one indexed step gathers (B*Q*K KiB) fit in L2: consecutive steps cycle
+    # through independently seeded index lists whose rows together exceed it
+    idx_sets = [idx]
+    if wl.mode == "indexed":
+        K_idx = wl.indices.shape[2]
+        n_sets = max(1, math.ceil(L2_BYTES * 2 / (B * Q * K_idx * 1024)))
+        for r in range(1, n_sets):
+            idx_sets.append(torch.from_numpy(synth.index_lists(B, Q, K_idx, wl.seq_lens,
+                                                               seed=1000 * (rank + 1) + r)).to(device))
+    idx_turn = [0]
     ws = m.new_workspace(B, Q)
     qt = torch.empty(B, Q, 64, 512, dtype=torch.bfloat16, device=device)
     o = torch.empty(B, Q, 64, 512, dtype=torch.bfloat16, device=device)
@@ -408,7 +459,9 @@ def main(argv=None):
         elif wl.mode == "paged":
             m.mla_attend_paged(qt, cache, table, lens, wl.scale, ws, o, lse, status)
         else:
-            m.mla_attend_indexed(qt, cache, idx, lens, wl.scale, ws, o, lse, status)
+            m.mla_attend_indexed(qt, cache, idx_sets[idx_turn[0] % len(idx_sets)], lens, wl.scale, ws, o, lse,
+                                 status)
+            idx_turn[0] += 1
 
     def up():
         m.mla_up_proj(o, w_uv, out)
@@ -418,7 +471,9 @@ def main(argv=None):
     torch.cuda.synchronize()
     assert int(status.item()) == 0, m.status_string(int(status.item()))
 
-    clocks = ClockSampler(local)
+    props = torch.cuda.get_device_properties(local)
+    bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+    clocks = ClockSampler(local, bus)
     clocks.start()
     time.sleep(0.3)
     K = args.steps
@@ -450,6 +505,19 @@ def main(argv=None):
     stage = [sum(ev[k][j].elapsed_time(ev[k][j + 1]) for k in range(Kb)) / Kb for j in range(3)]
     stage = reduce_max(stage, device)
     launches = K * 4  # absorb, attend, split-L combine, up-projection
+    # the attend + combine launches alone, back to back on the same stream: the duration
+    # of the pair as it runs inside the step (chained, nothing serialising it), for the
+    # roofline; the per-stage pass above puts events between the stages, which serialises
+    # every launch and adds its start-up to the stage
+    Ka = max(20, min(K, 400))
+    a_start, a_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a_start.record()
+    for _ in range(Ka):
+        attend()
+    a_stop.record()
+    torch.cuda.synchronize()
+    att_ms = reduce_max([a_start.elapsed_time(a_stop) / Ka], device)[0]
 
     # end to end through the public API with host buffers: H2D inputs, D2H output per step
     Ke = max(1, min(args.e2e_steps, K))
@@ -471,7 +539,12 @@ def main(argv=None):
     assert int(status.item()) == 0, m.status_string(int(status.item()))
 
     peaks, peak_kind = load_peaks()
-    att_gbs = acc["cache"] / (stage[1] * 1e-3) / 1e9
+    if wl.mode == "indexed":
+        l2_note = ("inputs larger than L2: steps cycle through %d seeded index lists, %.0f MB of gathered rows "
+                   "per cycle" % (len(idx_sets), len(idx_sets) * acc["cache"] / 1e6))
+    else:
+        l2_note = "inputs larger than L2 (cache %.0f MB per rank)" % (acc["cache"] / 1e6)
+    att_gbs = acc["cache"] / (att_ms * 1e-3) / 1e9
     src_hash = kernel_source_hash()
     traffic = TRAFFIC.get((args.config, src_hash))
     roofline = {"bound": "hbm", "achieved": att_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -480,7 +553,7 @@ def main(argv=None):
     t_mem = acc["cache"] / (peaks["hbm_gbs"] * 1e9)
     t_tc = acc["flops_attend"] / (peaks["bf16_tflops"] * 1e12)
     if t_tc > t_mem:
-        ach = acc["flops_attend"] / (stage[1] * 1e-3) / 1e12
+        ach = acc["flops_attend"] / (att_ms * 1e-3) / 1e12
         roofline = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                     "frac": ach / peaks["bf16_tflops"], "traffic": traffic,
                     "kernel": "attend_kernel + combine_kernel (mla_attend_*)", "peak_source": peak_kind}
@@ -492,9 +565,9 @@ def main(argv=None):
         "config": {"workload": args.config, "B": B, "q_len": Q, "mode": wl.mode,
                    "cache_rows": int(sum(int(x) for x in wl.seq_lens)) if wl.mode != "indexed" else None,
                    "heads": 64, "head_dim": 256, "latent": 512, "parallelism": f"dp{world} (independent batches)",
-                   "l2": "inputs larger than L2 (cache %.0f MB per rank)" % (acc["cache"] / 1e6)},
-        "stages_ms": {"absorb_q": stage[0], "attend": stage[1], "up_proj": stage[2]},
-        "attend_tflops": acc["flops_attend"] / (stage[1] * 1e-3) / 1e12,
+                   "l2": l2_note},
+        "stages_ms": {"absorb_q": stage[0], "attend": stage[1], "up_proj": stage[2], "attend_chained": att_ms},
+        "attend_tflops": acc["flops_attend"] / (att_ms * 1e-3) / 1e12,
         "roofline": roofline,
         "e2e": {"value": e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e_ms, "steps": Ke},
