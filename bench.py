@@ -39,8 +39,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one attend launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
 # ncu capture summarised in profiles/, keyed by the hash of the kernel source it was taken on.
 TRAFFIC = {
-    ("dense_decode", "14d6ff085e50bf20"): 277_809_920,
-    ("mtp_verify", "14d6ff085e50bf20"): 556_551_680,
+    ("dense_decode", "2f78743fc2d4f68e"): 277_555_968,
+    ("mtp_verify", "2f78743fc2d4f68e"): 556_532_480,
 }
 
 
