@@ -85,6 +85,23 @@ def step_bytes(wl) -> dict:
             "flops_total": flops_attend + flops_proj}
 
 
+def attend_roofline(acc, att_ms, peaks, peak_kind, traffic):
+    """Roofline of attend + combine: bound by whichever of the cache bytes at the HBM peak
+    and the attend FLOPs at the bf16 tensor peak takes longer; achieved = that quantity
+    over the measured duration ``att_ms`` (milliseconds)."""
+    t_mem = acc["cache"] / (peaks["hbm_gbs"] * 1e9)
+    t_tc = acc["flops_attend"] / (peaks["bf16_tflops"] * 1e12)
+    common = {"traffic": traffic, "kernel": "attend_kernel + combine_kernel (mla_attend_*)",
+              "peak_source": peak_kind}
+    if t_tc > t_mem:
+        ach = acc["flops_attend"] / (att_ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16_tflops"], **common}
+    ach = acc["cache"] / (att_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": ach / peaks["hbm_gbs"], **common}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -544,19 +561,8 @@ def main(argv=None):
                    "per cycle" % (len(idx_sets), len(idx_sets) * acc["cache"] / 1e6))
     else:
         l2_note = "inputs larger than L2 (cache %.0f MB per rank)" % (acc["cache"] / 1e6)
-    att_gbs = acc["cache"] / (att_ms * 1e-3) / 1e9
     src_hash = kernel_source_hash()
-    traffic = TRAFFIC.get((args.config, src_hash))
-    roofline = {"bound": "hbm", "achieved": att_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": att_gbs / peaks["hbm_gbs"], "traffic": traffic,
-                "kernel": "attend_kernel + combine_kernel (mla_attend_*)", "peak_source": peak_kind}
-    t_mem = acc["cache"] / (peaks["hbm_gbs"] * 1e9)
-    t_tc = acc["flops_attend"] / (peaks["bf16_tflops"] * 1e12)
-    if t_tc > t_mem:
-        ach = acc["flops_attend"] / (att_ms * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": ach / peaks["bf16_tflops"], "traffic": traffic,
-                    "kernel": "attend_kernel + combine_kernel (mla_attend_*)", "peak_source": peak_kind}
+    roofline = attend_roofline(acc, att_ms, peaks, peak_kind, TRAFFIC.get((args.config, src_hash)))
 
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
