@@ -85,6 +85,28 @@ def step_bytes(wl) -> dict:
             "flops_total": flops_attend + flops_proj}
 
 
+def index_list_sets(wl) -> int:
+    """How many independently seeded index lists the indexed workload's steps cycle
+    through, so that the rows they gather together exceed L2 (twice over)."""
+    K = wl.indices.shape[2]
+    return max(1, math.ceil(L2_BYTES * 2 / (wl.B * wl.Q * K * 1024)))
+
+
+def arm_config(wl, name, world) -> dict:
+    """The workload description of a bench line (the same for both arms)."""
+    acc = step_bytes(wl)
+    if wl.mode == "indexed":
+        n = index_list_sets(wl)
+        l2 = ("inputs larger than L2: steps cycle through %d seeded index lists, %.0f MB of gathered rows "
+              "per cycle" % (n, n * acc["cache"] / 1e6))
+    else:
+        l2 = "inputs larger than L2 (cache %.0f MB per rank)" % (acc["cache"] / 1e6)
+    return {"workload": name, "B": wl.B, "q_len": wl.Q, "mode": wl.mode,
+            "cache_rows": int(sum(int(x) for x in wl.seq_lens)) if wl.mode != "indexed" else None,
+            "heads": 64, "head_dim": 256, "latent": 512, "parallelism": f"dp{world} (independent batches)",
+            "l2": l2}
+
+
 def attend_roofline(acc, att_ms, peaks, peak_kind, traffic):
     """Roofline of attend + combine: bound by whichever of the cache bytes at the HBM peak
     and the attend FLOPs at the bf16 tensor peak takes longer; achieved = that quantity
@@ -322,7 +344,7 @@ def run_reference(args, wl_name):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl_name, "sample": sample},
+        "config": arm_config(wl, wl_name, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads_used(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
@@ -454,8 +476,7 @@ def main(argv=None):
     idx_sets = [idx]
     if wl.mode == "indexed":
         K_idx = wl.indices.shape[2]
-        n_sets = max(1, math.ceil(L2_BYTES * 2 / (B * Q * K_idx * 1024)))
-        for r in range(1, n_sets):
+        for r in range(1, index_list_sets(wl)):
             idx_sets.append(torch.from_numpy(synth.index_lists(B, Q, K_idx, wl.seq_lens,
                                                                seed=1000 * (rank + 1) + r)).to(device))
     idx_turn = [0]
@@ -556,11 +577,6 @@ def main(argv=None):
     assert int(status.item()) == 0, m.status_string(int(status.item()))
 
     peaks, peak_kind = load_peaks()
-    if wl.mode == "indexed":
-        l2_note = ("inputs larger than L2: steps cycle through %d seeded index lists, %.0f MB of gathered rows "
-                   "per cycle" % (len(idx_sets), len(idx_sets) * acc["cache"] / 1e6))
-    else:
-        l2_note = "inputs larger than L2 (cache %.0f MB per rank)" % (acc["cache"] / 1e6)
     src_hash = kernel_source_hash()
     roofline = attend_roofline(acc, att_ms, peaks, peak_kind, TRAFFIC.get((args.config, src_hash)))
 
@@ -568,10 +584,7 @@ def main(argv=None):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded SplitMix64/Box-Muller; random-init weights of the stated shapes)",
-        "config": {"workload": args.config, "B": B, "q_len": Q, "mode": wl.mode,
-                   "cache_rows": int(sum(int(x) for x in wl.seq_lens)) if wl.mode != "indexed" else None,
-                   "heads": 64, "head_dim": 256, "latent": 512, "parallelism": f"dp{world} (independent batches)",
-                   "l2": l2_note},
+        "config": arm_config(wl, args.config, world),
         "stages_ms": {"absorb_q": stage[0], "attend": stage[1], "up_proj": stage[2], "attend_chained": att_ms},
         "attend_tflops": acc["flops_attend"] / (att_ms * 1e-3) / 1e12,
         "roofline": roofline,
