@@ -113,6 +113,41 @@ def test_cache_bookkeeping_and_timeout_aid_reject_host_errors(lib):
     assert lib.mla_debug_wait_timeout(0, p, None) == m.MLA_ERR_ARG
 
 
+def test_kpool_entry_points_reject_host_errors(lib):
+    """Every case below returns before any device call."""
+    p, odd = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 4)
+    keys = lib.mla_kpool_keys  # (cache, seq_lens, B, R, Lmax, pool, pooled, stream)
+    assert keys(None, None, 1, 512, 64, 4, p, None) == m.MLA_ERR_ARG
+    assert keys(p, None, 1, 512, 64, 4, None, None) == m.MLA_ERR_ARG
+    assert keys(p, None, 0, 512, 64, 4, p, None) == m.MLA_ERR_ARG
+    assert keys(p, None, 1, 512, 0, 4, p, None) == m.MLA_ERR_ARG
+    assert keys(p, None, 1, 512, 64, 0, p, None) == m.MLA_ERR_ARG
+    assert keys(p, None, 1, 256, 64, 4, p, None) == m.MLA_ERR_UNSUPPORTED
+    assert keys(odd, None, 1, 512, 64, 4, p, None) == m.MLA_ERR_UNSUPPORTED
+    assert keys(p, None, 1, 512, 64, 4, odd, None) == m.MLA_ERR_UNSUPPORTED
+    assert keys(p, None, 1, 512, 3, 4, p, None) == m.MLA_OK  # no complete pool: nothing to launch
+
+    sel = lib.mla_kpool_select  # (pooled, w_query, seq_lens, B, Q, R, Lmax, pool, topk, tail, indices, W, stream)
+
+    def call(pooled=p, wq=p, B=1, Q=1, R=512, L=1024, pool=4, topk=16, tail=1, idx=p, W=None):
+        W = topk + (pool - 1 if tail else 0) if W is None else W
+        return sel(pooled, wq, None, B, Q, R, L, pool, topk, tail, idx, W, None)
+
+    assert call(pooled=None) == m.MLA_ERR_ARG
+    assert call(wq=None) == m.MLA_ERR_ARG
+    assert call(idx=None) == m.MLA_ERR_ARG
+    assert call(B=0) == m.MLA_ERR_ARG and call(Q=0) == m.MLA_ERR_ARG
+    assert call(L=0) == m.MLA_ERR_ARG and call(pool=0) == m.MLA_ERR_ARG
+    assert call(R=576) == m.MLA_ERR_UNSUPPORTED
+    assert call(topk=2) == m.MLA_ERR_ARG            # fewer positions than one pool
+    assert call(topk=18) == m.MLA_ERR_ARG           # not whole pools
+    assert call(pool=1, topk=1025) == m.MLA_ERR_ARG  # more chosen pools than the list holds
+    assert call(W=16) == m.MLA_ERR_ARG              # with a tail the width is topk + pool - 1
+    assert call(tail=0, W=19) == m.MLA_ERR_ARG      # without one it is topk
+    assert call(pooled=odd) == m.MLA_ERR_UNSUPPORTED
+    assert call(pool=1, topk=16, L=64 * 1024) == m.MLA_ERR_UNSUPPORTED  # pooled scores exceed shared memory
+
+
 def test_product_path_does_not_touch_oracle():
     """The binding and kernels never import the oracle (test infrastructure only)."""
     pkg = os.path.join(ROOT, "mla_absorbed_latent_mtp_b200")
