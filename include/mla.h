@@ -91,7 +91,8 @@ mla_status mla_attend_dense(const uint16_t *q_tilde, const uint16_t *cache, cons
  * Same as mla_attend_dense over a paged cache: logical row j of sequence b is
  *   pool[page_table[b * max_pages + j / page_size]][j % page_size][:].
  *   pool       [num_pages, page_size, R] bf16
- *   page_table [B, max_pages] int32   entries for pages past the end are ignored
+ *   page_table [B, max_pages] int32   entries for pages past the end are ignored;
+ *                                     max_pages * page_size and num_pages * page_size < 2^31
  *   seq_lens   [B] int32 (required)   0 <= L_b <= max_pages * page_size
  * page_size must be 64.  A used entry outside [0, num_pages) sets MLA_ERR_INDEX.
  * The result is bit-identical to mla_attend_dense on the same logical rows.

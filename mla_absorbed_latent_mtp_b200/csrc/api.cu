@@ -91,6 +91,7 @@ static mla_status attend_common(int mode, const uint16_t *q_tilde, const uint16_
     if (page_size != kPageTokens) return MLA_ERR_UNSUPPORTED;
     if (max_pages < 1 || num_pages < 1) return MLA_ERR_ARG;
     if ((long long)num_pages * kPageTokens >= (1LL << 31)) return MLA_ERR_ARG;
+    if ((long long)max_pages * kPageTokens >= (1LL << 31)) return MLA_ERR_ARG;  // positions are int32
   } else {
     if (Lmax < 1 || (long long)B * Lmax >= (1LL << 31)) return MLA_ERR_ARG;
   }
@@ -247,6 +248,7 @@ mla_status mla_debug_gather(int mode, const uint16_t *src, const int32_t *page_t
   if (src == nullptr || req == nullptr || out == nullptr || n_req < 0 || B < 1 || R < 1) return MLA_ERR_ARG;
   if (mode < 0 || mode > 2) return MLA_ERR_ARG;
   if (mode == mla::kModePaged && (page_table == nullptr || max_pages < 1 || num_pages < 1)) return MLA_ERR_ARG;
+  if (mode == mla::kModePaged && (long long)max_pages * mla::kPageTokens >= (1LL << 31)) return MLA_ERR_ARG;
   if (mode == mla::kModeIndexed && (indices == nullptr || K < 1 || Q < 1)) return MLA_ERR_ARG;
   if (mode != mla::kModePaged && Lmax < 1) return MLA_ERR_ARG;
   if (n_req == 0) return MLA_OK;

@@ -76,6 +76,11 @@ def test_paged_and_indexed_reject_host_errors(lib):
         m.MLA_ERR_ARG
     assert g(GOOD, GOOD, GOOD, GOOD, 1, 1, 64, 512, 32, 4, 4, 0.0625, GOOD, 1 << 30, GOOD, None, None, None) == \
         m.MLA_ERR_UNSUPPORTED
+    # positions are int32: a sequence of max_pages * 64 >= 2^31 rows, or a pool that size, is refused
+    assert g(GOOD, GOOD, GOOD, GOOD, 1, 1, 64, 512, 64, 1 << 25, 4, 0.0625, GOOD, 1 << 30, GOOD, None, None, None) == \
+        m.MLA_ERR_ARG
+    assert g(GOOD, GOOD, GOOD, GOOD, 1, 1, 64, 512, 64, 4, 1 << 25, 0.0625, GOOD, 1 << 30, GOOD, None, None, None) == \
+        m.MLA_ERR_ARG
     h = lib.mla_attend_indexed
     assert h(GOOD, GOOD, None, None, 1, 1, 64, 512, 8, 4, 0.0625, GOOD, 1 << 30, GOOD, None, None, None) == \
         m.MLA_ERR_ARG
@@ -95,6 +100,7 @@ def test_debug_gather_rejects_host_errors(lib):
     f = lib.mla_debug_gather
     assert f(3, GOOD, None, None, 1, 1, 512, 8, 0, 0, 0, GOOD, 1, GOOD, None, None) == m.MLA_ERR_ARG
     assert f(1, GOOD, None, None, 1, 1, 512, 8, 0, 0, 0, GOOD, 1, GOOD, None, None) == m.MLA_ERR_ARG
+    assert f(1, GOOD, GOOD, None, 1, 1, 512, 8, 1 << 25, 4, 0, GOOD, 1, GOOD, None, None) == m.MLA_ERR_ARG
     assert f(0, GOOD, None, None, 1, 1, 512, 8, 0, 0, 0, GOOD, 0, GOOD, None, None) == m.MLA_OK
 
 
