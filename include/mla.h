@@ -200,7 +200,8 @@ mla_status mla_cache_truncate_paged(uint16_t *pool, const int32_t *page_table, i
  *     then -1 up to topk; with_tail != 0 appends the positions of the incomplete pool up
  *     to t, then -1 up to W = topk + pool - 1 (W = topk without the tail).
  *   w_query [B, Q, R] bf16.  topk a positive multiple of pool, topk / pool <= 1024,
- *   Lmax / pool <= 51200.  The list feeds mla_attend_indexed with K = W (-1 entries unused).
+ *   Lmax / pool <= 51200, B * Q < 2^31 (mla_kpool_keys: B <= 65535).  The list feeds
+ *   mla_attend_indexed with K = W (-1 entries unused).
  */
 mla_status mla_kpool_keys(const uint16_t *cache, const int32_t *seq_lens, int B, int R, int Lmax, int pool,
                           float *pooled, void *stream);

@@ -219,6 +219,7 @@ mla_status mla_kpool_keys(const uint16_t *cache, const int32_t *seq_lens, int B,
   using namespace mla;
   if (cache == nullptr || pooled == nullptr || B < 1 || Lmax < 1 || pool < 1) return MLA_ERR_ARG;
   if (R != kLatent) return MLA_ERR_UNSUPPORTED;
+  if (B > 65535) return MLA_ERR_UNSUPPORTED;  // one grid row per sequence
   if (!kpool::aligned16(cache) || !kpool::aligned16(pooled)) return MLA_ERR_UNSUPPORTED;
   const int max_pools = Lmax / pool;
   if (max_pools < 1) return MLA_OK;
@@ -233,6 +234,7 @@ mla_status mla_kpool_select(const float *pooled, const uint16_t *w_query, const 
   using namespace mla;
   if (pooled == nullptr || w_query == nullptr || indices == nullptr || B < 1 || Q < 1 || Lmax < 1 || pool < 1)
     return MLA_ERR_ARG;
+  if ((long long)B * Q >= (1LL << 31)) return MLA_ERR_ARG;  // one block per query row
   if (R != kLatent) return MLA_ERR_UNSUPPORTED;
   if (topk < pool || topk % pool != 0 || topk / pool > kpool::kMaxChosen) return MLA_ERR_ARG;
   if (W != topk + (with_tail ? pool - 1 : 0)) return MLA_ERR_ARG;

@@ -131,6 +131,7 @@ def test_kpool_entry_points_reject_host_errors(lib):
     assert keys(p, None, 1, 256, 64, 4, p, None) == m.MLA_ERR_UNSUPPORTED
     assert keys(odd, None, 1, 512, 64, 4, p, None) == m.MLA_ERR_UNSUPPORTED
     assert keys(p, None, 1, 512, 64, 4, odd, None) == m.MLA_ERR_UNSUPPORTED
+    assert keys(p, None, 65536, 512, 64, 4, p, None) == m.MLA_ERR_UNSUPPORTED  # grid rows
     assert keys(p, None, 1, 512, 3, 4, p, None) == m.MLA_OK  # no complete pool: nothing to launch
 
     sel = lib.mla_kpool_select  # (pooled, w_query, seq_lens, B, Q, R, Lmax, pool, topk, tail, indices, W, stream)
@@ -143,6 +144,7 @@ def test_kpool_entry_points_reject_host_errors(lib):
     assert call(wq=None) == m.MLA_ERR_ARG
     assert call(idx=None) == m.MLA_ERR_ARG
     assert call(B=0) == m.MLA_ERR_ARG and call(Q=0) == m.MLA_ERR_ARG
+    assert call(B=1 << 16, Q=1 << 15) == m.MLA_ERR_ARG  # B * Q query rows overflow the grid
     assert call(L=0) == m.MLA_ERR_ARG and call(pool=0) == m.MLA_ERR_ARG
     assert call(R=576) == m.MLA_ERR_UNSUPPORTED
     assert call(topk=2) == m.MLA_ERR_ARG            # fewer positions than one pool
