@@ -1,16 +1,20 @@
 #!/usr/bin/env python
-"""Throughput of the absorbed-MLA decode path on B200.
+"""Throughput of the absorbed-MLA decode and verify path on B200.
 
-One step = the whole hot path over one batch of the dense decode workload (B=32
-sequences, q_len=1, 8192 cached latent rows each, 64 heads, 256-dim NoPE heads, latent
-512, bf16, seed 0): query absorption (q~ = W_UK^T q), split-L latent attention with the
-log-sum-exp combine, and the W_UV up-projection.  ``value`` is the effective HBM
-bandwidth of a step: the algorithmic bytes (every visible cache row read once, 1,024 B,
-plus both weight matrices, q, and the output) divided by the device time of a step;
-with N ranks every rank runs its own batch (weak scaling, no collective on the data
-path) and value sums the bytes over ranks divided by the slowest rank's time.
+One step = the whole hot path over one batch of a workload: query absorption
+(q~ = W_UK^T q), split-L latent attention with the log-sum-exp combine, and the W_UV
+up-projection (64 heads, 256-dim NoPE heads, latent 512, bf16).  The five workloads are
+tiny dense decode (B=1, 256 rows), dense decode (B=32, 8,192 rows), MTP verify (B=16,
+q_len=6, 32,768 + 6 rows), ragged paged decode (B=64, 1,024..131,072 rows in 64-row pages)
+and indexed sparse decode (B=32, 2,048 listed rows of 131,072).  One JSON line reports
+them all under "configs"; its headline fields are those of ragged paged decode, the
+largest.  ``value`` is the effective HBM bandwidth of a step: the algorithmic bytes (every
+visible cache row read once, 1,024 B, plus both weight matrices, q, and the output)
+divided by the device time of a step; with N ranks every rank runs its own batch (weak
+scaling, no collective on the data path) and value sums the bytes over ranks divided by
+the slowest rank's time.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME|all]
 
 ``--impl reference`` times the fp64 CPU oracle (test infrastructure) on a bounded sample
 of the same workload instead; it is the reported CPU baseline.
@@ -50,13 +54,19 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="dense_decode")
+    ap.add_argument("--config", default="all",
+                    help="one workload name, or 'all' (every configuration; the headline is ragged paged decode)")
     ap.add_argument("--e2e-steps", type=int, default=100)
-    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU-oracle sample")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0,
+                    help="budget of the CPU-oracle samples, shared by the configurations")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--next-rows", action="store_true",
                     help="time the cache bookkeeping and k-pool producer entry points instead")
     ap.add_argument("--kpool-seqs", type=int, default=4, help="sequences of 131,072 rows for --next-rows")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="profiling size: override the batch of the selected configuration")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="profiling size: every sequence gets this many rows (paged: instead of ragged lengths)")
     return ap.parse_args(argv)
 
 
@@ -278,15 +288,21 @@ def aggregate(local_ms, local_bytes, device):
 
 # ----------------------------------------------------------------------------- CPU oracle baseline
 
-def cpu_baseline(wl, budget_s):
+def cpu_baseline(wl, budget_s, got=None):
     """Time the fp64 oracle (expanded form, as it stands) on a bounded sample: heads of
-    sequence 0, query 0, added until the budget is spent.  Reported in the metric's unit."""
-    import numpy as np  # noqa: F401
+    sequence 0, query 0, added until the budget is spent.  Reported in the metric's unit.
+
+    ``got`` (the GPU step's output bits, [B, Q, 64, 256]) is compared with the oracle on the
+    same sample: max-abs and mean-abs error (the parity gate's quantities) and max-abs over
+    the RMS of the reference (a relative measure that does not shrink with the output)."""
+    import numpy as np
     import oracle
     t_start = time.perf_counter()
     heads = 0
+    outs = []
     while heads < 64:
-        oracle.reference(wl, pairs=[(0, 0)], heads=[heads], row_source=None)
+        r = oracle.reference(wl, pairs=[(0, 0)], heads=[heads], row_source=None)
+        outs.append(r[(0, 0)]["out"][0])
         heads += 1
         if time.perf_counter() - t_start > budget_s:
             break
@@ -294,9 +310,19 @@ def cpu_baseline(wl, budget_s):
     L = int(wl.seq_lens[0]) if wl.mode != "indexed" else wl.indices.shape[2]
     bytes_attributed = L * 1024 * heads / 64.0
     cores = threads_used()
-    return {"value": bytes_attributed / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"sequence 0, query 0, {heads} of 64 heads, {L} cached rows, expanded fp64 form "
-                      f"({dt:.1f} s)"}
+    res = {"value": bytes_attributed / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
+           "sample": f"sequence 0, query 0, {heads} of 64 heads, {L} cached rows, expanded fp64 form "
+                     f"({dt:.1f} s)"}
+    if got is not None:
+        ref = np.stack(outs)
+        g = (np.asarray(got, dtype=np.uint16)[0, 0, :heads].astype(np.uint32) << 16).view(np.float32)
+        err = np.abs(g.astype(np.float64) - ref)
+        rms = float(np.sqrt((ref ** 2).mean()))
+        res["parity"] = {"max_abs": float(err.max()), "mean_abs": float(err.mean()),
+                         "max_abs_over_rms": float(err.max()) / rms if rms > 0 else None,
+                         "gate": "max-abs <= 2e-2 and mean-abs <= 2e-3",
+                         "pass": bool(err.max() <= 2e-2 and err.mean() <= 2e-3)}
+    return res
 
 
 def threads_used():
@@ -422,39 +448,32 @@ def run_next_rows(args):
     }))
 
 
-def main(argv=None):
-    args = parse_args(argv)
-    world, rank, local = dist_env()
-    if args.next_rows:
-        if rank == 0:
-            run_next_rows(args)
-        return
-    if args.impl == "reference":
-        # under torchrun rank 0 alone runs the oracle; the other ranks exit without work
-        # (no process group: nothing is exchanged)
-        run_reference(args, args.config)
-        return
+CONFIG_NAMES = ("tiny_dense_decode", "dense_decode", "mtp_verify", "ragged_paged_decode", "indexed_sparse_decode")
+# the largest of the five workloads that fit one GPU: the line's headline
+HEADLINE = "ragged_paged_decode"
+# host->device bytes the end-to-end leg may copy per configuration (a few seconds of PCIe)
+E2E_BYTES_CAP = 24e9
 
+
+def _seq_len(name, args):
+    """Rows per sequence for a profiling-size run (MTP verify: prefix + the 6 window rows)."""
+    if args.seq_len is None:
+        return None
+    return args.seq_len + (6 if name == "mtp_verify" else 0)
+
+
+def measure_config(name, args, device, rank, world, clocks, peaks, peak_kind, src_hash, cpu_seconds):
+    """One configuration: the timed steps, the stage breakdown, the chained attend timing for
+    the roofline, the end-to-end leg with host buffers, and (rank 0 of a 1-GPU run) the CPU
+    oracle on a sample, whose outputs are also compared with this run's.  Returns the
+    configuration's record; every rank takes the same collective steps."""
     import numpy as np
     import torch
 
     import mla_absorbed_latent_mtp_b200 as m
     import synth
 
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
-
-    from mla_absorbed_latent_mtp_b200 import _build
-    if rank == 0:
-        _build.build()
-    barrier()
-    m.lib()
-
-    wl = synth.make_workload(args.config, seed=rank, with_data=False)
+    wl = synth.make_workload(name, seed=rank, with_data=False, B=args.batch, L=_seq_len(name, args))
     acc = step_bytes(wl)
     B, Q = wl.B, wl.Q
 
@@ -509,11 +528,6 @@ def main(argv=None):
     torch.cuda.synchronize()
     assert int(status.item()) == 0, m.status_string(int(status.item()))
 
-    props = torch.cuda.get_device_properties(local)
-    bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
-    clocks = ClockSampler(local, bus)
-    clocks.start()
-    time.sleep(0.3)
     K = args.steps
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
@@ -528,8 +542,6 @@ def main(argv=None):
     torch.cuda.synchronize()
     wall1 = time.time()
     barrier()
-    time.sleep(0.1)
-    clocks.stop()
     local_ms = start.elapsed_time(stop) / K
     ms, value = aggregate(local_ms, acc["total"], device)
     # per-stage breakdown in a separate pass: events between the stages serialise them
@@ -550,18 +562,20 @@ def main(argv=None):
     Ka = max(20, min(K, 400))
     a_start, a_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
+    aw0 = time.time()
     a_start.record()
     for _ in range(Ka):
         attend()
     a_stop.record()
     torch.cuda.synchronize()
+    aw1 = time.time()
     att_ms = reduce_max([a_start.elapsed_time(a_stop) / Ka], device)[0]
 
     # end to end through the public API with host buffers: H2D inputs, D2H output per step
-    Ke = max(1, min(args.e2e_steps, K))
-    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     h2d = host_cache.numel() * 2 + host_q.numel() * 2 + host_lens.numel() * 4
     d2h = host_out.numel() * 2
+    Ke = max(1, min(args.e2e_steps, K, int(E2E_BYTES_CAP // h2d)))
+    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e_start.record()
@@ -576,29 +590,106 @@ def main(argv=None):
     e_ms, e_value = aggregate(e_start.elapsed_time(e_stop) / Ke, acc["total"], device)
     assert int(status.item()) == 0, m.status_string(int(status.item()))
 
-    peaks, peak_kind = load_peaks()
-    src_hash = kernel_source_hash()
-    roofline = attend_roofline(acc, att_ms, peaks, peak_kind, TRAFFIC.get((args.config, src_hash)))
-
-    result = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded SplitMix64/Box-Muller; random-init weights of the stated shapes)",
-        "config": arm_config(wl, args.config, world),
+    roofline = attend_roofline(acc, att_ms, peaks, peak_kind, TRAFFIC.get((name, src_hash)))
+    label = name if args.batch is None and args.seq_len is None else \
+        f"{name} at a profiling size (B={B}, rows={args.seq_len})"
+    rec = {
+        "workload": arm_config(wl, label, world),
+        "value": value, "unit": UNIT, "ms_per_step": ms, "steps": K,
         "stages_ms": {"absorb_q": stage[0], "attend": stage[1], "up_proj": stage[2], "attend_chained": att_ms},
         "attend_tflops": acc["flops_attend"] / (att_ms * 1e-3) / 1e12,
+        "attend_cache_bytes": acc["cache"], "attend_flops": acc["flops_attend"],
         "roofline": roofline,
         "e2e": {"value": e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e_ms, "steps": Ke},
         "gpu_launches": launches,
         "clocks": clocks.summary(wall0, wall1),
-        "kernel_src": src_hash,
+        "clocks_attend_chained": clocks.summary(aw0, aw1),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        wl_cpu = synth.make_workload(args.config, with_data=False)
+    if cpu_seconds > 0:
+        if wl.mode == "indexed":
+            # one more step on the workload's own index lists, whose output the sample checks
+            idx_turn[0] = 0
+            absorb(); attend(); up()
+            torch.cuda.synchronize()
+        wl_cpu = synth.make_workload(name, with_data=False, B=args.batch, L=_seq_len(name, args))
         wl_cpu.cache = host_cache.numpy().view(np.uint16) if wl.mode != "paged" else None
         wl_cpu.pool = host_cache.numpy().view(np.uint16) if wl.mode == "paged" else None
-        result["cpu_baseline"] = cpu_baseline(wl_cpu, args.cpu_seconds)
+        host_out.copy_(out.view(torch.int16))  # the last timed step's output (same inputs every step)
+        got = host_out.numpy().view(np.uint16)
+        rec["cpu_baseline"] = cpu_baseline(wl_cpu, cpu_seconds, got)
+    del cache, host_cache, idx_sets, ws
+    torch.cuda.empty_cache()
+    return rec
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_env()
+    if args.next_rows:
+        if rank == 0:
+            run_next_rows(args)
+        return
+    names = list(CONFIG_NAMES) if args.config == "all" else [args.config]
+    headline = HEADLINE if args.config == "all" else args.config
+    if args.impl == "reference":
+        # under torchrun rank 0 alone runs the oracle; the other ranks exit without work
+        # (no process group: nothing is exchanged)
+        run_reference(args, headline)
+        return
+
+    import torch
+
+    import mla_absorbed_latent_mtp_b200 as m
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    from mla_absorbed_latent_mtp_b200 import _build
+    if rank == 0:
+        _build.build()
+    barrier()
+    m.lib()
+
+    props = torch.cuda.get_device_properties(local)
+    bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+    clocks = ClockSampler(local, bus)
+    clocks.start()
+    time.sleep(0.3)
+    peaks, peak_kind = load_peaks()
+    src_hash = kernel_source_hash()
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    per_cfg = {}
+    for name in names:
+        per_cfg[name] = measure_config(name, args, device, rank, world, clocks, peaks, peak_kind, src_hash,
+                                       args.cpu_seconds / len(names) if want_cpu else 0.0)
+    time.sleep(0.1)
+    clocks.stop()
+
+    head = per_cfg[headline]
+    result = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded SplitMix64/Box-Muller; random-init weights of the stated shapes)",
+        "config": head["workload"],
+        "stages_ms": head["stages_ms"],
+        "attend_tflops": head["attend_tflops"],
+        "roofline": head["roofline"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+        "kernel_src": src_hash,
+        "peaks": {k: peaks.get(k) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")},
+        "configs": {n: {k: v for k, v in r.items() if k != "workload"} | {"config": r["workload"]}
+                    for n, r in per_cfg.items()},
+    }
+    if "cpu_baseline" in head:
+        result["cpu_baseline"] = head["cpu_baseline"]
     if rank == 0:
         print(json.dumps(result))
     if world > 1:

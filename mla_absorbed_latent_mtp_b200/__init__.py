@@ -95,9 +95,39 @@ def _check(fn, code):
 
 
 def _check_cuda(*tensors):
+    dev = None
     for t in tensors:
-        if t is not None and not t.is_cuda:
+        if t is None:
+            continue
+        if not t.is_cuda:
             raise ValueError("tensors must be CUDA tensors")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors must be on one device ({dev} and {t.device})")
+
+
+def _require(t, name, dtype, shape=None, min_numel=None, optional=False):
+    """Refuse, before any pointer reaches the C ABI, a tensor whose dtype, layout or size
+    would let a kernel read or write outside it: the kernels address memory only from the
+    pointer and the sizes passed, so a strided, narrower or smaller tensor must never get
+    that far.  ``shape`` may hold None for a free dimension."""
+    import torch
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    want = {"bf16": torch.bfloat16, "i32": torch.int32, "f32": torch.float32, "u8": torch.uint8}[dtype]
+    if t.dtype != want:
+        raise ValueError(f"{name} must be {want}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None:
+        if t.dim() != len(shape) or any(w is not None and int(g) != int(w) for g, w in zip(t.shape, shape)):
+            raise ValueError(f"{name} must have shape {tuple('*' if w is None else w for w in shape)}, "
+                             f"got {tuple(t.shape)}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name} needs at least {min_numel} elements, got {t.numel()}")
 
 
 # ----------------------------------------------------------------------------- entry points
@@ -116,8 +146,13 @@ def new_workspace(B: int, Q: int):
 def mla_absorb_q(q, w_uk, q_tilde=None, stream=None):
     """q [n, H, D] or [B, Q, H, D] bf16, w_uk [H, D, R] bf16 -> q_tilde [..., H, R] bf16."""
     import torch
-    _check_cuda(q, w_uk, q_tilde)
+    _require(q, "q", "bf16")
+    if q.dim() < 3 or tuple(q.shape[-2:]) != (H, D):
+        raise ValueError(f"q must be [..., {H}, {D}], got {tuple(q.shape)}")
+    _require(w_uk, "w_uk", "bf16", (H, D, R))
     n = q.numel() // (H * D)
+    _require(q_tilde, "q_tilde", "bf16", tuple(q.shape[:-1]) + (R,), optional=True)
+    _check_cuda(q, w_uk, q_tilde)
     if q_tilde is None:
         q_tilde = torch.empty(*q.shape[:-1], R, dtype=torch.bfloat16, device=q.device)
     _check("mla_absorb_q", lib().mla_absorb_q(_ptr(q), _ptr(w_uk), _ptr(q_tilde), n, H, D, R, _stream(stream)))
@@ -127,12 +162,30 @@ def mla_absorb_q(q, w_uk, q_tilde=None, stream=None):
 def mla_up_proj(o_latent, w_uv, out=None, stream=None):
     """o_latent [..., H, R] bf16, w_uv [H, D, R] bf16 -> out [..., H, D] bf16."""
     import torch
-    _check_cuda(o_latent, w_uv, out)
+    _require(o_latent, "o_latent", "bf16")
+    if o_latent.dim() < 3 or tuple(o_latent.shape[-2:]) != (H, R):
+        raise ValueError(f"o_latent must be [..., {H}, {R}], got {tuple(o_latent.shape)}")
+    _require(w_uv, "w_uv", "bf16", (H, D, R))
     n = o_latent.numel() // (H * R)
+    _require(out, "out", "bf16", tuple(o_latent.shape[:-1]) + (D,), optional=True)
+    _check_cuda(o_latent, w_uv, out)
     if out is None:
         out = torch.empty(*o_latent.shape[:-1], D, dtype=torch.bfloat16, device=o_latent.device)
     _check("mla_up_proj", lib().mla_up_proj(_ptr(o_latent), _ptr(w_uv), _ptr(out), n, H, D, R, _stream(stream)))
     return out
+
+
+def _check_attend(q_tilde, workspace, o_latent, lse, status, seq_lens, seq_lens_required=False):
+    """Common checks of the attend calls; returns (B, Q)."""
+    _require(q_tilde, "q_tilde", "bf16", (None, None, H, R))
+    B, Q = int(q_tilde.shape[0]), int(q_tilde.shape[1])
+    _require(seq_lens, "seq_lens", "i32", min_numel=B, optional=not seq_lens_required)
+    if workspace is not None:
+        _require(workspace, "workspace", "u8", min_numel=mla_attend_workspace_bytes(B, Q))
+    _require(o_latent, "o_latent", "bf16", (B, Q, H, R), optional=True)
+    _require(lse, "lse", "f32", (B, Q, H), optional=True)
+    _require(status, "status", "i32", min_numel=1, optional=True)
+    return B, Q
 
 
 def _attend_outputs(q_tilde, o_latent, lse, want_lse):
@@ -148,8 +201,11 @@ def _attend_outputs(q_tilde, o_latent, lse, want_lse):
 def mla_attend_dense(q_tilde, cache, seq_lens=None, scale=SCALE, workspace=None, o_latent=None, lse=None,
                      status=None, want_lse=True, stream=None):
     """q_tilde [B, Q, H, R], cache [B, Lmax, R] (bf16), seq_lens [B] int32 or None."""
+    B, Q = _check_attend(q_tilde, workspace, o_latent, lse, status, seq_lens)
+    _require(cache, "cache", "bf16", (None, None, R))
+    if cache.shape[0] < B:
+        raise ValueError(f"cache holds {cache.shape[0]} sequences, q_tilde {B}")
     _check_cuda(q_tilde, cache, seq_lens, workspace, o_latent, lse, status)
-    B, Q = q_tilde.shape[0], q_tilde.shape[1]
     Lmax = cache.shape[1]
     workspace = new_workspace(B, Q) if workspace is None else workspace
     o_latent, lse = _attend_outputs(q_tilde, o_latent, lse, want_lse)
@@ -163,8 +219,11 @@ def mla_attend_dense_noalloc(q_tilde, cache, seq_lens=None, scale=SCALE, o_laten
                              want_lse=True, stream=None):
     """mla_attend_dense without a workspace argument: for callers that cannot allocate
     device memory, the scratch is a fixed 32 MiB array inside the library (see mla.h)."""
+    B, Q = _check_attend(q_tilde, None, o_latent, lse, status, seq_lens)
+    _require(cache, "cache", "bf16", (None, None, R))
+    if cache.shape[0] < B:
+        raise ValueError(f"cache holds {cache.shape[0]} sequences, q_tilde {B}")
     _check_cuda(q_tilde, cache, seq_lens, o_latent, lse, status)
-    B, Q = q_tilde.shape[0], q_tilde.shape[1]
     o_latent, lse = _attend_outputs(q_tilde, o_latent, lse, want_lse)
     _check("mla_attend_dense_noalloc", lib().mla_attend_dense_noalloc(
         _ptr(q_tilde), _ptr(cache), _ptr(seq_lens), B, Q, H, R, cache.shape[1], scale, _ptr(o_latent), _ptr(lse),
@@ -175,8 +234,12 @@ def mla_attend_dense_noalloc(q_tilde, cache, seq_lens=None, scale=SCALE, o_laten
 def mla_attend_paged(q_tilde, pool, page_table, seq_lens, scale=SCALE, workspace=None, o_latent=None, lse=None,
                      status=None, want_lse=True, stream=None):
     """pool [P, 64, R] bf16, page_table [B, max_pages] int32, seq_lens [B] int32."""
+    B, Q = _check_attend(q_tilde, workspace, o_latent, lse, status, seq_lens, seq_lens_required=True)
+    _require(pool, "pool", "bf16", (None, PAGE, R))
+    _require(page_table, "page_table", "i32", (None, None))
+    if page_table.shape[0] < B:
+        raise ValueError(f"page_table has {page_table.shape[0]} rows, q_tilde {B} sequences")
     _check_cuda(q_tilde, pool, page_table, seq_lens, workspace, o_latent, lse, status)
-    B, Q = q_tilde.shape[0], q_tilde.shape[1]
     workspace = new_workspace(B, Q) if workspace is None else workspace
     o_latent, lse = _attend_outputs(q_tilde, o_latent, lse, want_lse)
     _check("mla_attend_paged", lib().mla_attend_paged(
@@ -189,8 +252,12 @@ def mla_attend_paged(q_tilde, pool, page_table, seq_lens, scale=SCALE, workspace
 def mla_attend_indexed(q_tilde, cache, indices, seq_lens=None, scale=SCALE, workspace=None, o_latent=None, lse=None,
                        status=None, want_lse=True, stream=None):
     """cache [B, Lmax, R] bf16, indices [B, Q, K] int32."""
+    B, Q = _check_attend(q_tilde, workspace, o_latent, lse, status, seq_lens)
+    _require(cache, "cache", "bf16", (None, None, R))
+    if cache.shape[0] < B:
+        raise ValueError(f"cache holds {cache.shape[0]} sequences, q_tilde {B}")
+    _require(indices, "indices", "i32", (B, Q, None))
     _check_cuda(q_tilde, cache, indices, seq_lens, workspace, o_latent, lse, status)
-    B, Q = q_tilde.shape[0], q_tilde.shape[1]
     workspace = new_workspace(B, Q) if workspace is None else workspace
     o_latent, lse = _attend_outputs(q_tilde, o_latent, lse, want_lse)
     _check("mla_attend_indexed", lib().mla_attend_indexed(
@@ -203,6 +270,11 @@ def mla_attend_indexed(q_tilde, cache, indices, seq_lens=None, scale=SCALE, work
 def mla_debug_gather(mode, src, req, page_table=None, indices=None, B=None, Q=1, Lmax=0, status=None, stream=None):
     """Rows the attend kernels would address for requests req [n, 3] int32 (b, i, k)."""
     import torch
+    _require(src, "src", "bf16", (None, None, R))
+    _require(req, "req", "i32", (None, 3))
+    _require(page_table, "page_table", "i32", (None, None), optional=mode != MODE_PAGED)
+    _require(indices, "indices", "i32", (None, None, None), optional=mode != MODE_INDEXED)
+    _require(status, "status", "i32", min_numel=1, optional=True)
     _check_cuda(src, req, page_table, indices, status)
     n = req.shape[0]
     out = torch.empty(n, R, dtype=torch.bfloat16, device=src.device)
@@ -218,16 +290,29 @@ def mla_debug_gather(mode, src, req, page_table=None, indices=None, B=None, Q=1,
 def mla_cache_append_dense(cache, seq_lens, rows, status=None, stream=None):
     """Append rows [B, Q, R] bf16 at positions seq_lens[b] + i of cache [B, Lmax, R];
     seq_lens [B] int32 advances by Q (in place)."""
-    _check_cuda(cache, seq_lens, rows, status)
+    _require(rows, "rows", "bf16", (None, None, R))
     B, Q = rows.shape[0], rows.shape[1]
+    _require(cache, "cache", "bf16", (None, None, R))
+    if cache.shape[0] < B:
+        raise ValueError(f"cache holds {cache.shape[0]} sequences, rows {B}")
+    _require(seq_lens, "seq_lens", "i32", min_numel=B)
+    _require(status, "status", "i32", min_numel=1, optional=True)
+    _check_cuda(cache, seq_lens, rows, status)
     _check("mla_cache_append_dense", lib().mla_cache_append_dense(
         _ptr(cache), _ptr(seq_lens), _ptr(rows), B, Q, R, cache.shape[1], _ptr(status), _stream(stream)))
 
 
 def mla_cache_append_paged(pool, page_table, seq_lens, rows, status=None, stream=None):
     """Append rows [B, Q, R] bf16 through page_table [B, max_pages] into pool [P, 64, R]."""
-    _check_cuda(pool, page_table, seq_lens, rows, status)
+    _require(rows, "rows", "bf16", (None, None, R))
     B, Q = rows.shape[0], rows.shape[1]
+    _require(pool, "pool", "bf16", (None, PAGE, R))
+    _require(page_table, "page_table", "i32", (None, None))
+    if page_table.shape[0] < B:
+        raise ValueError(f"page_table has {page_table.shape[0]} rows, rows {B} sequences")
+    _require(seq_lens, "seq_lens", "i32", min_numel=B)
+    _require(status, "status", "i32", min_numel=1, optional=True)
+    _check_cuda(pool, page_table, seq_lens, rows, status)
     _check("mla_cache_append_paged", lib().mla_cache_append_paged(
         _ptr(pool), _ptr(page_table), _ptr(seq_lens), _ptr(rows), B, Q, R, pool.shape[1], page_table.shape[1],
         pool.shape[0], _ptr(status), _stream(stream)))
@@ -235,6 +320,12 @@ def mla_cache_append_paged(pool, page_table, seq_lens, rows, status=None, stream
 
 def mla_cache_truncate_dense(cache, seq_lens, keep, q_len, status=None, stream=None):
     """Keep the first keep[b] of the last q_len rows of each sequence; zero the rest."""
+    _require(seq_lens, "seq_lens", "i32", (None,))
+    _require(keep, "keep", "i32", min_numel=seq_lens.shape[0])
+    _require(cache, "cache", "bf16", (None, None, R))
+    if cache.shape[0] < seq_lens.shape[0]:
+        raise ValueError(f"cache holds {cache.shape[0]} sequences, seq_lens {seq_lens.shape[0]}")
+    _require(status, "status", "i32", min_numel=1, optional=True)
     _check_cuda(cache, seq_lens, keep, status)
     _check("mla_cache_truncate_dense", lib().mla_cache_truncate_dense(
         _ptr(cache), _ptr(seq_lens), _ptr(keep), seq_lens.shape[0], q_len, R, cache.shape[1], _ptr(status),
@@ -243,6 +334,13 @@ def mla_cache_truncate_dense(cache, seq_lens, keep, q_len, status=None, stream=N
 
 def mla_cache_truncate_paged(pool, page_table, seq_lens, keep, q_len, status=None, stream=None):
     """Paged counterpart of mla_cache_truncate_dense."""
+    _require(seq_lens, "seq_lens", "i32", (None,))
+    _require(keep, "keep", "i32", min_numel=seq_lens.shape[0])
+    _require(pool, "pool", "bf16", (None, PAGE, R))
+    _require(page_table, "page_table", "i32", (None, None))
+    if page_table.shape[0] < seq_lens.shape[0]:
+        raise ValueError(f"page_table has {page_table.shape[0]} rows, seq_lens {seq_lens.shape[0]}")
+    _require(status, "status", "i32", min_numel=1, optional=True)
     _check_cuda(pool, page_table, seq_lens, keep, status)
     _check("mla_cache_truncate_paged", lib().mla_cache_truncate_paged(
         _ptr(pool), _ptr(page_table), _ptr(seq_lens), _ptr(keep), seq_lens.shape[0], q_len, R, pool.shape[1],
@@ -251,6 +349,7 @@ def mla_cache_truncate_paged(pool, page_table, seq_lens, keep, q_len, status=Non
 
 def mla_debug_wait_timeout(limit_cycles, status, stream=None):
     """Run the pipeline's bounded wait on a barrier nothing completes (test aid)."""
+    _require(status, "status", "i32", min_numel=1)
     _check_cuda(status)
     _check("mla_debug_wait_timeout", lib().mla_debug_wait_timeout(int(limit_cycles), _ptr(status), _stream(stream)))
 
@@ -258,8 +357,13 @@ def mla_debug_wait_timeout(limit_cycles, status, stream=None):
 def mla_kpool_keys(cache, pool, seq_lens=None, pooled=None, stream=None):
     """Pooled keys [B, Lmax // pool, R] fp32 of every complete pool of cache [B, Lmax, R]."""
     import torch
-    _check_cuda(cache, seq_lens, pooled)
+    _require(cache, "cache", "bf16", (None, None, R))
     B, Lmax = cache.shape[0], cache.shape[1]
+    _require(seq_lens, "seq_lens", "i32", min_numel=B, optional=True)
+    if pool < 1:
+        raise ValueError("pool must be positive")
+    _require(pooled, "pooled", "f32", (B, Lmax // pool, R), optional=True)
+    _check_cuda(cache, seq_lens, pooled)
     if pooled is None:
         pooled = torch.zeros(B, Lmax // pool, R, dtype=torch.float32, device=cache.device)
     _check("mla_kpool_keys", lib().mla_kpool_keys(_ptr(cache), _ptr(seq_lens), B, R, Lmax, pool, _ptr(pooled),
@@ -270,9 +374,16 @@ def mla_kpool_keys(cache, pool, seq_lens=None, pooled=None, stream=None):
 def mla_kpool_select(pooled, w_query, pool, topk, seq_lens=None, with_tail=True, Lmax=None, stream=None):
     """Index lists [B, Q, topk (+ pool - 1)] int32 for w_query [B, Q, R] bf16."""
     import torch
-    _check_cuda(pooled, w_query, seq_lens)
+    _require(w_query, "w_query", "bf16", (None, None, R))
     B, Q = w_query.shape[0], w_query.shape[1]
+    _require(pooled, "pooled", "f32", (B, None, R))
+    _require(seq_lens, "seq_lens", "i32", min_numel=B, optional=True)
+    if pool < 1:
+        raise ValueError("pool must be positive")
     Lmax = pooled.shape[1] * pool if Lmax is None else Lmax
+    if Lmax // pool > pooled.shape[1]:
+        raise ValueError(f"pooled holds {pooled.shape[1]} pools per sequence, Lmax {Lmax} needs {Lmax // pool}")
+    _check_cuda(pooled, w_query, seq_lens)
     W = topk + (pool - 1 if with_tail else 0)
     out = torch.empty(B, Q, W, dtype=torch.int32, device=w_query.device)
     _check("mla_kpool_select", lib().mla_kpool_select(

@@ -11,6 +11,26 @@ MAX_ABS_TOL = 2e-2
 MEAN_ABS_TOL = 2e-3
 
 
+def decode_bf16(u: int) -> float:
+    """Value of one bfloat16 bit pattern, decoded field by field (IEEE 754 binary16-brain:
+    1 sign bit, 8 exponent bits with bias 127, 7 fraction bits), independently of the
+    oracle's array widening."""
+    u = int(u) & 0xFFFF
+    sign = -1.0 if u & 0x8000 else 1.0
+    exp = (u >> 7) & 0xFF
+    frac = u & 0x7F
+    if exp == 0xFF:
+        return sign * math.inf if frac == 0 else math.nan
+    if exp == 0:  # zero or subnormal: frac * 2^-133
+        return sign * math.ldexp(frac, -126 - 7)
+    return sign * math.ldexp(128 + frac, exp - 127 - 7)
+
+
+def decode_list(bits):
+    """Flat list of Python floats for an array of bfloat16 bit patterns."""
+    return [decode_bf16(x) for x in np.asarray(bits).ravel()]
+
+
 def errors(got, ref):
     err = np.abs(np.asarray(got, dtype=np.float64) - np.asarray(ref, dtype=np.float64))
     return float(err.max()) if err.size else 0.0, float(err.mean()) if err.size else 0.0

@@ -10,7 +10,7 @@ import torch
 import oracle
 import synth
 from conftest import read_golden
-from helpers import gate, errors, tiny_workload
+from helpers import decode_list, gate, errors, tiny_workload
 
 
 # ----------------------------------------------------------------------------- page facts
@@ -38,8 +38,7 @@ def test_dimensions_match_page():
 
 def _brute_force(wl):
     """Pure-Python loops: expanded keys/values, softmax, weighted sum (tiny shapes only)."""
-    def f(bits):
-        return [float(x) for x in oracle.widen(np.asarray(bits)).ravel()]
+    f = decode_list  # bits decoded field by field, not through oracle.widen
 
     H, D, R = wl.q.shape[2], wl.q.shape[3], wl.w_uk.shape[2]
     out = {}
