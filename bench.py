@@ -63,6 +63,8 @@ def parse_args(argv=None):
     ap.add_argument("--next-rows", action="store_true",
                     help="time the cache bookkeeping and k-pool producer entry points instead")
     ap.add_argument("--kpool-seqs", type=int, default=4, help="sequences of 131,072 rows for --next-rows")
+    ap.add_argument("--prefill-lengths", default="1024,4096",
+                    help="prefill lengths for the expanded-vs-absorbed comparison ('' to skip)")
     ap.add_argument("--batch", type=int, default=None,
                     help="profiling size: override the batch of the selected configuration")
     ap.add_argument("--seq-len", type=int, default=None,
@@ -555,6 +557,43 @@ def measure_config(name, args, device, rank, world, clocks, peaks, peak_kind, sr
     stage = [sum(ev[k][j].elapsed_time(ev[k][j + 1]) for k in range(Kb)) / Kb for j in range(3)]
     stage = reduce_max(stage, device)
     launches = K * 4  # absorb, attend, split-L combine, up-projection
+    # the same step with the up-projection fused into the split-L merge (mla_attend_up_*):
+    # absorb, attend, merge + up-projection
+    def attend_up():
+        if wl.mode == "dense":
+            m.mla_attend_up_dense(qt, cache, w_uv, lens, wl.scale, ws, out, None, lse, status)
+        elif wl.mode == "paged":
+            m.mla_attend_up_paged(qt, cache, table, lens, w_uv, wl.scale, ws, out, None, lse, status)
+        else:
+            m.mla_attend_up_indexed(qt, cache, idx_sets[idx_turn[0] % len(idx_sets)], w_uv, lens, wl.scale, ws, out,
+                                    None, lse, status)
+            idx_turn[0] += 1
+
+    for _ in range(args.warmup):
+        absorb(); attend_up()
+    f_start, f_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    f_start.record()
+    for _ in range(K):
+        absorb(); attend_up()
+    f_stop.record()
+    torch.cuda.synchronize()
+    fused_ms, fused_value = aggregate(f_start.elapsed_time(f_stop) / K, acc["total"], device)
+    # the attend kernel and the fused merge + up-projection alone, back to back
+    Kf = max(20, min(K, 400))
+    k_start, k_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    k_start.record()
+    for _ in range(Kf):
+        attend_up()
+    k_stop.record()
+    torch.cuda.synchronize()
+    attend_up_ms = reduce_max([k_start.elapsed_time(k_stop) / Kf], device)[0]
+    # the step the line reports: whichever path (chained or fused) is faster on this workload
+    best = "fused" if fused_ms < ms else "chained"
+    if best == "fused":
+        launches = K * 3  # absorb, attend, merge + up-projection
     # the attend + combine launches alone, back to back on the same stream: the duration
     # of the pair as it runs inside the step (chained, nothing serialising it), for the
     # roofline; the per-stage pass above puts events between the stages, which serialises
@@ -583,7 +622,10 @@ def measure_config(name, args, device, rank, world, clocks, peaks, peak_kind, sr
         cache.view(torch.int16).copy_(host_cache, non_blocking=True)
         q.view(torch.int16).copy_(host_q, non_blocking=True)
         lens.copy_(host_lens, non_blocking=True)
-        absorb(); attend(); up()
+        if best == "fused":
+            absorb(); attend_up()
+        else:
+            absorb(); attend(); up()
         host_out.copy_(out.view(torch.int16), non_blocking=True)
     e_stop.record()
     torch.cuda.synchronize()
@@ -595,7 +637,13 @@ def measure_config(name, args, device, rank, world, clocks, peaks, peak_kind, sr
         f"{name} at a profiling size (B={B}, rows={args.seq_len})"
     rec = {
         "workload": arm_config(wl, label, world),
-        "value": value, "unit": UNIT, "ms_per_step": ms, "steps": K,
+        "value": fused_value if best == "fused" else value, "unit": UNIT,
+        "ms_per_step": fused_ms if best == "fused" else ms, "steps": K, "step_path": best,
+        "paths": {"chained": {"ms_per_step": ms, "value": value,
+                              "kernels": "absorb, attend, split-L combine, up-projection"},
+                  "fused": {"ms_per_step": fused_ms, "value": fused_value,
+                            "kernels": "absorb, attend, split-L merge fused with the up-projection",
+                            "attend_and_merge_up_ms": attend_up_ms}},
         "stages_ms": {"absorb_q": stage[0], "attend": stage[1], "up_proj": stage[2], "attend_chained": att_ms},
         "attend_tflops": acc["flops_attend"] / (att_ms * 1e-3) / 1e12,
         "attend_cache_bytes": acc["cache"], "attend_flops": acc["flops_attend"],
@@ -621,6 +669,83 @@ def measure_config(name, args, device, rank, world, clocks, peaks, peak_kind, sr
     del cache, host_cache, idx_sets, ws
     torch.cuda.empty_cache()
     return rec
+
+
+def prefill_flops(L, B=1):
+    """Algorithmic FLOPs of one causal prefill of B sequences of L tokens (64 heads, head 256,
+    latent 512): causal (query, key) pairs L(L+1)/2 per sequence and head."""
+    H, D, R = 64, 256, 512
+    pairs = B * L * (L + 1) // 2
+    expand = 2 * (2 * B * L * R * H * D)          # k and v from the latents
+    attn_expanded = pairs * H * 2 * (2 * D)       # q.k and p.v over 256-wide heads
+    proj = 2 * (2 * B * L * H * D * R)            # absorb q and up-project o
+    attn_absorbed = pairs * H * 2 * (2 * R)       # q~.c and p.c over the 512-wide latent
+    return {"expanded": expand + attn_expanded, "absorbed": proj + attn_absorbed,
+            "expanded_attention": attn_expanded, "absorbed_attention": attn_absorbed}
+
+
+def measure_prefill(lengths, device, peaks, reps=5):
+    """Module 05 section 5's comparison on B200: one causal prefill of L tokens in the
+    expanded form (mla_expand_kv + mla_prefill_expanded) and in the absorbed form
+    (mla_absorb_q + mla_attend_dense with q_len = L + mla_up_proj), timed with CUDA events
+    (warm-up first, median of `reps`)."""
+    import numpy as np
+    import torch
+
+    import mla_absorbed_latent_mtp_b200 as m
+    import synth
+
+    res = []
+    for L in lengths:
+        wl = synth.make_workload(mode="dense", B=1, Q=L, L=L, with_data=True, seed=5)
+        dev = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(  # noqa: E731
+            torch.bfloat16)
+        q, wk, wv, cache = dev(wl.q), dev(wl.w_uk), dev(wl.w_uv), dev(wl.cache)
+        lens = torch.from_numpy(wl.seq_lens).to(device)
+        st = torch.zeros(1, dtype=torch.int32, device=device)
+        k = torch.empty(1, L, 64, 256, dtype=torch.bfloat16, device=device)
+        v = torch.empty_like(k)
+        out_e = torch.empty_like(k)
+        qt = torch.empty(1, L, 64, 512, dtype=torch.bfloat16, device=device)
+        o = torch.empty_like(qt)
+        out_a = torch.empty_like(k)
+        ws = m.new_workspace(1, L)
+
+        def expanded():
+            m.mla_expand_kv(cache[0], wk, wv, k[0], v[0])
+            m.mla_prefill_expanded(q, k, v, wl.scale, out_e, want_lse=False, status=st)
+
+        def absorbed():
+            m.mla_absorb_q(q, wk, qt)
+            m.mla_attend_dense(qt, cache, lens, wl.scale, ws, o, None, st, want_lse=False)
+            m.mla_up_proj(o, wv, out_a)
+
+        def timed(fn):
+            for _ in range(2):
+                fn()
+            ts = []
+            for _ in range(reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(); fn(); b.record()
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b))
+            return float(np.median(ts))
+
+        te, ta = timed(expanded), timed(absorbed)
+        assert int(st.item()) == 0, m.status_string(int(st.item()))
+        diff = float((out_e.float() - out_a.float()).abs().max())
+        fl = prefill_flops(L)
+        peak = peaks["bf16_tflops"]
+        res.append({"L": L, "B": 1,
+                    "expanded": {"ms": te, "flops": fl["expanded"], "tflops": fl["expanded"] / (te * 1e-3) / 1e12,
+                                 "frac_of_tensor_peak": fl["expanded"] / (te * 1e-3) / 1e12 / peak},
+                    "absorbed": {"ms": ta, "flops": fl["absorbed"], "tflops": fl["absorbed"] / (ta * 1e-3) / 1e12,
+                                 "frac_of_tensor_peak": fl["absorbed"] / (ta * 1e-3) / 1e12 / peak},
+                    "faster": "expanded" if te < ta else "absorbed", "speedup": max(te, ta) / min(te, ta),
+                    "max_abs_difference_between_forms": diff})
+        del k, v, out_e, qt, o, out_a, ws, q, cache
+        torch.cuda.empty_cache()
+    return res
 
 
 def main(argv=None):
@@ -667,6 +792,10 @@ def main(argv=None):
     for name in names:
         per_cfg[name] = measure_config(name, args, device, rank, world, clocks, peaks, peak_kind, src_hash,
                                        args.cpu_seconds / len(names) if want_cpu else 0.0)
+    prefill = None
+    if args.prefill_lengths:
+        lengths = [int(x) for x in args.prefill_lengths.split(",") if x]
+        prefill = measure_prefill(lengths, device, peaks)
     time.sleep(0.1)
     clocks.stop()
 
@@ -690,6 +819,8 @@ def main(argv=None):
     }
     if "cpu_baseline" in head:
         result["cpu_baseline"] = head["cpu_baseline"]
+    if prefill is not None:
+        result["prefill_comparison"] = prefill
     if rank == 0:
         print(json.dumps(result))
     if world > 1:

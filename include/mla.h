@@ -30,6 +30,12 @@
  *    MLA_OK, so the first error is kept; the caller zeroes it and reads it after its
  *    own synchronisation.  Outputs are unspecified when *status != MLA_OK.
  *  - Supported sizes in this version: H = 64, D = 256, R = 512.
+ *  - Launch chaining: each kernel may start while the previous kernel on the stream is
+ *    still running and waits for it (griddepcontrol.wait) before it reads that kernel's
+ *    results.  The one exception is the projection weights: mla_absorb_q and mla_up_proj
+ *    start streaming w_uk / w_uv before that wait, so the weights must not be written by
+ *    the kernel launched immediately before them on the same stream.  Weights written
+ *    earlier (or on another stream followed by an event wait, or by a memcpy) are safe.
  */
 #ifndef MLA_B200_H
 #define MLA_B200_H
@@ -127,17 +133,76 @@ mla_status mla_up_proj(const uint16_t *o_latent, const uint16_t *w_uv, uint16_t 
                        int n, int H, int D, int R, void *stream);
 
 /*
+ * Attention with the value up-projection fused into its split-L merge, Module 05 section 3:
+ * "the latent-space sum is expanded once, at the end" -- out_h = U_h^V o_h with
+ * o_h = sum_j a_j c_j, computed without o making a round trip through global memory.
+ * Same inputs and semantics as mla_attend_dense / _paged / _indexed, plus
+ *   w_uv     [H, D, R] bf16   U^V per head (as for mla_up_proj), D = 256
+ *   out      [B, Q, H, D] bf16  the attention output (what mla_up_proj returns)
+ *   o_latent [B, Q, H, R] bf16 or NULL: also store the normalised latent output
+ *   lse      [B, Q, H] fp32 or NULL
+ * The workspace is the same as the unfused call's (mla_attend_workspace_bytes).  The merge
+ * and the projection run in one kernel launched after the attend kernel: clusters of four
+ * CTAs per head split the latent into chunks of 128, merge their chunk of the partials
+ * into the tensor-core operand and sum the four partial products through distributed
+ * shared memory.  w_uv is read before that kernel waits for the attend kernel (see the
+ * launch-chaining note above).  Results match mla_attend_* followed by mla_up_proj to
+ * rounding (here o is rounded to bf16 per 128-wide chunk, exactly as mla_up_proj's input).
+ */
+mla_status mla_attend_up_dense(const uint16_t *q_tilde, const uint16_t *cache, const int32_t *seq_lens, int B, int Q,
+                               int H, int R, int Lmax, float scale, const uint16_t *w_uv, int D, void *workspace,
+                               size_t ws_bytes, uint16_t *out, uint16_t *o_latent, float *lse, int32_t *status,
+                               void *stream);
+mla_status mla_attend_up_paged(const uint16_t *q_tilde, const uint16_t *pool, const int32_t *page_table,
+                               const int32_t *seq_lens, int B, int Q, int H, int R, int page_size, int max_pages,
+                               int num_pages, float scale, const uint16_t *w_uv, int D, void *workspace,
+                               size_t ws_bytes, uint16_t *out, uint16_t *o_latent, float *lse, int32_t *status,
+                               void *stream);
+mla_status mla_attend_up_indexed(const uint16_t *q_tilde, const uint16_t *cache, const int32_t *indices,
+                                 const int32_t *seq_lens, int B, int Q, int H, int R, int Lmax, int K, float scale,
+                                 const uint16_t *w_uv, int D, void *workspace, size_t ws_bytes, uint16_t *out,
+                                 uint16_t *o_latent, float *lse, int32_t *status, void *stream);
+
+/*
+ * Prefill in the expanded form, Module 05 section 5 ("prefill and decode may want different
+ * algebra"): when every token of a sequence is a query, the pass is compute-heavy and the
+ * naive algebra -- expand keys and values once, then ordinary attention over 256-wide heads
+ * -- does half the attention arithmetic of the absorbed form (whose scores and value sums
+ * run over the 512-wide latent).  The absorbed form of the same prefill is
+ * mla_absorb_q -> mla_attend_dense (q_len = L, cache = the sequence's own latents) ->
+ * mla_up_proj; these two calls are the expanded one, for measuring which form wins.
+ *
+ * mla_expand_kv, Module 05 section 1: k[n, h, :] = U_h^K c[n, :], v[n, h, :] = U_h^V c[n, :].
+ *   c [n, R] bf16 latents; w_uk, w_uv [H, D, R] bf16; k, v [n, H, D] bf16 (fp32 accumulation).
+ * mla_prefill_expanded: causal attention of B sequences of L tokens over themselves,
+ *   out[b, t, h, :] = sum_{j <= t} softmax_j(scale * q[b, t, h] . k[b, j, h]) v[b, j, h]
+ *   q, k, v, out [B, L, H, D] bf16 (token-major, as mla_expand_kv writes k and v with
+ *   n = B * L); lse [B, L, H] fp32 natural-log sum-exp or NULL.  k and v must be finite
+ *   (rows past a sequence's last query are read but weighted zero).  B * L * H < 2^31.
+ */
+mla_status mla_expand_kv(const uint16_t *c, const uint16_t *w_uk, const uint16_t *w_uv, uint16_t *k, uint16_t *v,
+                         int n, int H, int D, int R, void *stream);
+mla_status mla_prefill_expanded(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int L, int H, int D,
+                                float scale, uint16_t *out, float *lse, int32_t *status, void *stream);
+
+/*
  * mla_attend_dense for callers that cannot allocate device memory (for example a plugin
  * inside a host runtime that owns all device memory and passes its plugins no workspace,
  * or a runtime whose memory plan is fixed at start-up).  There is no counterpart on the
  * pages: it is a packaging variant of mla_attend_dense, with the same arguments minus
  * the workspace and the same results.
- *  - Scratch comes from a 32 MiB array inside the library, held by every GPU that loads
- *    the library until the process exits.  Sizes whose mla_attend_workspace_bytes(B, Q, H, R)
- *    exceeds 32 MiB return MLA_ERR_WORKSPACE and enqueue nothing.
- *  - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
- *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- *    with that device current; make that first call before any stream capture.
+ *  - Scratch comes from a 32 MiB array inside the library.  Sizes whose
+ *    mla_attend_workspace_bytes(B, Q, H, R) exceeds 32 MiB return MLA_ERR_WORKSPACE and
+ *    enqueue nothing.
+ *  - No call allocates: no cudaMalloc, cudaFree or allocating library call.  The array
+ *    itself is device memory that the CUDA runtime reserves when it loads the library's
+ *    code module holding it on a device.  With the default lazy module loading that
+ *    happens in the first call of this entry point on that device (which looks the array's
+ *    address up with cudaGetSymbolAddress, with that device current); it is then held
+ *    until the process exits.  A caller with a fixed memory plan makes that first call at
+ *    start-up, or sets CUDA_MODULE_LOADING=EAGER so that every device reserves the array
+ *    when the context is created.  If the reservation fails, the call returns MLA_ERR_CUDA.
+ *    Make the first call before any stream capture.
  *  - All calls share the one array, so calls whose kernels overlap on the GPU (different
  *    streams, or several host threads) race and corrupt each other's results; serialise
  *    them.  No part of the array has to start at zero.

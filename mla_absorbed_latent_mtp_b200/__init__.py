@@ -22,7 +22,8 @@ SCALE = 1.0 / 16.0
 EXPORTS = ("mla_status_string", "mla_last_error_string", "mla_absorb_q", "mla_attend_dense", "mla_attend_paged", "mla_attend_indexed",
            "mla_up_proj", "mla_attend_workspace_bytes", "mla_debug_gather", "mla_attend_dense_noalloc",
            "mla_cache_append_dense", "mla_cache_append_paged", "mla_cache_truncate_dense", "mla_cache_truncate_paged",
-           "mla_debug_wait_timeout", "mla_kpool_keys", "mla_kpool_select")
+           "mla_debug_wait_timeout", "mla_kpool_keys", "mla_kpool_select", "mla_attend_up_dense",
+           "mla_attend_up_paged", "mla_attend_up_indexed", "mla_expand_kv", "mla_prefill_expanded")
 
 
 class MLAError(RuntimeError):
@@ -65,11 +66,19 @@ def lib():
     L.mla_kpool_keys.restype = ctypes.c_int32
     L.mla_kpool_select.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
     L.mla_kpool_select.restype = ctypes.c_int32
+    L.mla_attend_up_dense.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, i32, vp, sz, vp, vp, vp, vp, vp]
+    L.mla_attend_up_paged.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, vp, i32, vp, sz, vp, vp,
+                                      vp, vp, vp]
+    L.mla_attend_up_indexed.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, i32, vp, sz, vp, vp, vp,
+                                        vp, vp]
+    L.mla_expand_kv.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
+    L.mla_prefill_expanded.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, vp]
     L.mla_debug_wait_timeout.argtypes = [ctypes.c_longlong, vp, vp]
     L.mla_debug_wait_timeout.restype = ctypes.c_int32
     for name in ("mla_absorb_q", "mla_up_proj", "mla_attend_dense", "mla_attend_paged", "mla_attend_indexed",
                  "mla_debug_gather", "mla_attend_dense_noalloc", "mla_cache_append_dense", "mla_cache_append_paged",
-                 "mla_cache_truncate_dense", "mla_cache_truncate_paged"):
+                 "mla_cache_truncate_dense", "mla_cache_truncate_paged", "mla_attend_up_dense", "mla_attend_up_paged",
+                 "mla_attend_up_indexed", "mla_expand_kv", "mla_prefill_expanded"):
         getattr(L, name).restype = ctypes.c_int32
     _lib = L
     return L
@@ -267,6 +276,112 @@ def mla_attend_indexed(q_tilde, cache, indices, seq_lens=None, scale=SCALE, work
     return o_latent, lse
 
 
+def _fused_outputs(q_tilde, w_uv, out, o_latent, lse, want_lse):
+    import torch
+    B, Q = q_tilde.shape[0], q_tilde.shape[1]
+    _require(w_uv, "w_uv", "bf16", (H, D, R))
+    _require(out, "out", "bf16", (B, Q, H, D), optional=True)
+    if out is None:
+        out = torch.empty(B, Q, H, D, dtype=torch.bfloat16, device=q_tilde.device)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Q, H, dtype=torch.float32, device=q_tilde.device)
+    return out, lse
+
+
+def mla_attend_up_dense(q_tilde, cache, w_uv, seq_lens=None, scale=SCALE, workspace=None, out=None, o_latent=None,
+                        lse=None, status=None, want_lse=True, stream=None):
+    """Attention over a contiguous cache with the W_UV up-projection fused into the split-L
+    merge: q_tilde [B, Q, H, R], cache [B, Lmax, R], w_uv [H, D, R] -> out [B, Q, H, D]
+    (and lse); o_latent [B, Q, H, R] is written too when given."""
+    B, Q = _check_attend(q_tilde, workspace, o_latent, lse, status, seq_lens)
+    _require(cache, "cache", "bf16", (None, None, R))
+    if cache.shape[0] < B:
+        raise ValueError(f"cache holds {cache.shape[0]} sequences, q_tilde {B}")
+    out, lse = _fused_outputs(q_tilde, w_uv, out, o_latent, lse, want_lse)
+    _check_cuda(q_tilde, cache, w_uv, seq_lens, workspace, out, o_latent, lse, status)
+    workspace = new_workspace(B, Q) if workspace is None else workspace
+    _check("mla_attend_up_dense", lib().mla_attend_up_dense(
+        _ptr(q_tilde), _ptr(cache), _ptr(seq_lens), B, Q, H, R, cache.shape[1], scale, _ptr(w_uv), D,
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), _ptr(o_latent), _ptr(lse),
+        _ptr(status), _stream(stream)))
+    return out, lse
+
+
+def mla_attend_up_paged(q_tilde, pool, page_table, seq_lens, w_uv, scale=SCALE, workspace=None, out=None,
+                        o_latent=None, lse=None, status=None, want_lse=True, stream=None):
+    """Paged counterpart of mla_attend_up_dense (pool [P, 64, R], page_table [B, max_pages])."""
+    B, Q = _check_attend(q_tilde, workspace, o_latent, lse, status, seq_lens, seq_lens_required=True)
+    _require(pool, "pool", "bf16", (None, PAGE, R))
+    _require(page_table, "page_table", "i32", (None, None))
+    if page_table.shape[0] < B:
+        raise ValueError(f"page_table has {page_table.shape[0]} rows, q_tilde {B} sequences")
+    out, lse = _fused_outputs(q_tilde, w_uv, out, o_latent, lse, want_lse)
+    _check_cuda(q_tilde, pool, page_table, seq_lens, w_uv, workspace, out, o_latent, lse, status)
+    workspace = new_workspace(B, Q) if workspace is None else workspace
+    _check("mla_attend_up_paged", lib().mla_attend_up_paged(
+        _ptr(q_tilde), _ptr(pool), _ptr(page_table), _ptr(seq_lens), B, Q, H, R, pool.shape[1], page_table.shape[1],
+        pool.shape[0], scale, _ptr(w_uv), D, _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out),
+        _ptr(o_latent), _ptr(lse), _ptr(status), _stream(stream)))
+    return out, lse
+
+
+def mla_attend_up_indexed(q_tilde, cache, indices, w_uv, seq_lens=None, scale=SCALE, workspace=None, out=None,
+                          o_latent=None, lse=None, status=None, want_lse=True, stream=None):
+    """Index-list counterpart of mla_attend_up_dense (indices [B, Q, K] int32)."""
+    B, Q = _check_attend(q_tilde, workspace, o_latent, lse, status, seq_lens)
+    _require(cache, "cache", "bf16", (None, None, R))
+    if cache.shape[0] < B:
+        raise ValueError(f"cache holds {cache.shape[0]} sequences, q_tilde {B}")
+    _require(indices, "indices", "i32", (B, Q, None))
+    out, lse = _fused_outputs(q_tilde, w_uv, out, o_latent, lse, want_lse)
+    _check_cuda(q_tilde, cache, indices, w_uv, seq_lens, workspace, out, o_latent, lse, status)
+    workspace = new_workspace(B, Q) if workspace is None else workspace
+    _check("mla_attend_up_indexed", lib().mla_attend_up_indexed(
+        _ptr(q_tilde), _ptr(cache), _ptr(indices), _ptr(seq_lens), B, Q, H, R, cache.shape[1], indices.shape[2],
+        scale, _ptr(w_uv), D, _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out),
+        _ptr(o_latent), _ptr(lse), _ptr(status), _stream(stream)))
+    return out, lse
+
+
+def mla_expand_kv(c, w_uk, w_uv, k=None, v=None, stream=None):
+    """Keys and values of every head from the latents: c [..., R] bf16 -> k, v [..., H, D]."""
+    import torch
+    _require(c, "c", "bf16")
+    if c.dim() < 1 or c.shape[-1] != R:
+        raise ValueError(f"c must be [..., {R}], got {tuple(c.shape)}")
+    _require(w_uk, "w_uk", "bf16", (H, D, R))
+    _require(w_uv, "w_uv", "bf16", (H, D, R))
+    n = c.numel() // R
+    shape = tuple(c.shape[:-1]) + (H, D)
+    _require(k, "k", "bf16", shape, optional=True)
+    _require(v, "v", "bf16", shape, optional=True)
+    _check_cuda(c, w_uk, w_uv, k, v)
+    k = torch.empty(shape, dtype=torch.bfloat16, device=c.device) if k is None else k
+    v = torch.empty(shape, dtype=torch.bfloat16, device=c.device) if v is None else v
+    _check("mla_expand_kv", lib().mla_expand_kv(_ptr(c), _ptr(w_uk), _ptr(w_uv), _ptr(k), _ptr(v), n, H, D, R,
+                                                _stream(stream)))
+    return k, v
+
+
+def mla_prefill_expanded(q, k, v, scale=SCALE, out=None, lse=None, status=None, want_lse=True, stream=None):
+    """Causal self-attention of B sequences of L tokens: q, k, v [B, L, H, D] bf16 -> out (and lse)."""
+    import torch
+    _require(q, "q", "bf16", (None, None, H, D))
+    B, L = int(q.shape[0]), int(q.shape[1])
+    _require(k, "k", "bf16", (B, L, H, D))
+    _require(v, "v", "bf16", (B, L, H, D))
+    _require(out, "out", "bf16", (B, L, H, D), optional=True)
+    _require(lse, "lse", "f32", (B, L, H), optional=True)
+    _require(status, "status", "i32", min_numel=1, optional=True)
+    _check_cuda(q, k, v, out, lse, status)
+    out = torch.empty(B, L, H, D, dtype=torch.bfloat16, device=q.device) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty(B, L, H, dtype=torch.float32, device=q.device)
+    _check("mla_prefill_expanded", lib().mla_prefill_expanded(
+        _ptr(q), _ptr(k), _ptr(v), B, L, H, D, scale, _ptr(out), _ptr(lse), _ptr(status), _stream(stream)))
+    return out, lse
+
+
 def mla_debug_gather(mode, src, req, page_table=None, indices=None, B=None, Q=1, Lmax=0, status=None, stream=None):
     """Rows the attend kernels would address for requests req [n, 3] int32 (b, i, k)."""
     import torch
@@ -393,11 +508,20 @@ def mla_kpool_select(pooled, w_query, pool, topk, seq_lens=None, with_tail=True,
 
 
 def mla_decode(q, w_uk, w_uv, cache, seq_lens=None, *, mode=MODE_DENSE, page_table=None, indices=None,
-               scale=SCALE, workspace=None, status=None, stream=None):
-    """The whole path: absorb -> attend (dense / paged / indexed) -> up-project.
+               scale=SCALE, workspace=None, status=None, stream=None, fused=False):
+    """The whole path: absorb -> attend (dense / paged / indexed) -> up-project.  With
+    fused=True the up-projection runs inside the split-L merge (mla_attend_up_*).
 
     q [B, Q, H, D] bf16 -> out [B, Q, H, D] bf16 (and lse [B, Q, H])."""
     qt = mla_absorb_q(q, w_uk, stream=stream)
+    if fused:
+        if mode == MODE_DENSE:
+            return mla_attend_up_dense(qt, cache, w_uv, seq_lens, scale, workspace, status=status, stream=stream)
+        if mode == MODE_PAGED:
+            return mla_attend_up_paged(qt, cache, page_table, seq_lens, w_uv, scale, workspace, status=status,
+                                       stream=stream)
+        return mla_attend_up_indexed(qt, cache, indices, w_uv, seq_lens, scale, workspace, status=status,
+                                     stream=stream)
     if mode == MODE_DENSE:
         o, lse = mla_attend_dense(qt, cache, seq_lens, scale, workspace, status=status, stream=stream)
     elif mode == MODE_PAGED:

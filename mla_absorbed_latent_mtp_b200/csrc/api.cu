@@ -58,6 +58,14 @@ int sm_count_for(int dev) {
   return cache[dev];
 }
 
+// W_UV[h][d][r] for the fused merge + up-projection: dims {R, D, H}, boxes of 64 r x 128 d.
+bool make_w_uv_map(CUtensorMap *map, const uint16_t *w_uv) {
+  const uint64_t dims[3] = {(uint64_t)kLatent, (uint64_t)kHeadDim, (uint64_t)kHeads};
+  const uint64_t strides[2] = {(uint64_t)kLatent * 2, (uint64_t)kHeadDim * kLatent * 2};
+  const uint32_t box[3] = {64, 128, 1};
+  return make_map(map, w_uv, 3, dims, strides, box);
+}
+
 }  // namespace
 
 static thread_local cudaError_t g_last_error = cudaSuccess;
@@ -77,14 +85,23 @@ int device_sm_count() {
 }
 
 // Shared validation and launch for the three attend modes.
+// Shared validation and launch for the three attend modes.  With w_uv / out given, the
+// split-L merge runs fused with the up-projection (o_latent optional); without, the combine
+// writes o_latent (required).
 static mla_status attend_common(int mode, const uint16_t *q_tilde, const uint16_t *cache, const int32_t *page_table,
                                 const int32_t *indices, const int32_t *seq_lens, int B, int Q, int H, int R, int Lmax,
                                 int page_size, int max_pages, int num_pages, int K, float scale, void *workspace,
-                                size_t ws_bytes, uint16_t *o_latent, float *lse, int32_t *status, void *stream) {
-  if (q_tilde == nullptr || cache == nullptr || o_latent == nullptr) return MLA_ERR_ARG;
+                                size_t ws_bytes, uint16_t *o_latent, float *lse, int32_t *status, void *stream,
+                                const uint16_t *w_uv = nullptr, int D = 0, uint16_t *out = nullptr) {
+  const bool fused = (w_uv != nullptr || out != nullptr);
+  if (q_tilde == nullptr || cache == nullptr) return MLA_ERR_ARG;
+  if (fused ? (w_uv == nullptr || out == nullptr) : (o_latent == nullptr)) return MLA_ERR_ARG;
+  if (fused && D != kHeadDim) return MLA_ERR_UNSUPPORTED;
+  if (fused && (!aligned16(w_uv) || !aligned16(out))) return MLA_ERR_UNSUPPORTED;
+  if (o_latent != nullptr && !aligned16(o_latent)) return MLA_ERR_UNSUPPORTED;
   if (B < 1 || Q < 1 || !isfinite(scale)) return MLA_ERR_ARG;
   if (H != kHeads || R != kLatent) return MLA_ERR_UNSUPPORTED;
-  if (!aligned16(q_tilde) || !aligned16(cache) || !aligned16(o_latent)) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(q_tilde) || !aligned16(cache)) return MLA_ERR_UNSUPPORTED;
   if ((long long)B * Q * H >= (1LL << 31)) return MLA_ERR_ARG;
   if (mode == kModePaged) {
     if (page_table == nullptr || seq_lens == nullptr) return MLA_ERR_ARG;
@@ -144,7 +161,12 @@ static mla_status attend_common(int mode, const uint16_t *q_tilde, const uint16_
   p.o_latent = o_latent;
   p.lse = lse;
   p.status = status;
-  return cuda_status(launch_attend(mode, tm_cache, tm_qt, p, reinterpret_cast<cudaStream_t>(stream)));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!fused) return cuda_status(launch_attend(mode, tm_cache, tm_qt, p, st));
+  CUtensorMap tm_w;
+  if (!make_w_uv_map(&tm_w, w_uv)) return cuda_status(cudaErrorInvalidValue);
+  if (cudaError_t e = launch_attend(mode, tm_cache, tm_qt, p, st, false); e != cudaSuccess) return cuda_status(e);
+  return cuda_status(launch_merge_up(tm_w, p, mode, out, st));
 }
 
 static mla_status proj_common(bool absorb, const uint16_t *x, const uint16_t *w, uint16_t *out, int n, int H, int D,
@@ -177,9 +199,66 @@ static mla_status proj_common(bool absorb, const uint16_t *x, const uint16_t *w,
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+static mla_status expand_common(const uint16_t *c, const uint16_t *w_uk, const uint16_t *w_uv, uint16_t *k, uint16_t *v,
+                                int n, int H, int D, int R, void *stream) {
+  if (c == nullptr || w_uk == nullptr || w_uv == nullptr || k == nullptr || v == nullptr) return MLA_ERR_ARG;
+  if (n < 1) return MLA_ERR_ARG;
+  if (H != kHeads || D != kHeadDim || R != kLatent) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(c) || !aligned16(w_uk) || !aligned16(w_uv) || !aligned16(k) || !aligned16(v))
+    return MLA_ERR_UNSUPPORTED;
+  if ((long long)n * H >= (1LL << 31)) return MLA_ERR_ARG;
+  const int n_tile = std::min(128, (n + 31) / 32 * 32);
+  CUtensorMap tm_wk, tm_wv, tm_x;
+  {
+    const uint64_t dims[3] = {(uint64_t)R, (uint64_t)D, (uint64_t)H};
+    const uint64_t strides[2] = {(uint64_t)R * 2, (uint64_t)D * R * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if (!make_map(&tm_wk, w_uk, 3, dims, strides, box) || !make_map(&tm_wv, w_uv, 3, dims, strides, box))
+      return cuda_status(cudaErrorInvalidValue);
+  }
+  {
+    // c[n][r] seen as X[n][1][r]: one row per token, shared by every head
+    const uint64_t dims[3] = {(uint64_t)R, 1, (uint64_t)n};
+    const uint64_t strides[2] = {(uint64_t)R * 2, (uint64_t)R * 2};
+    const uint32_t box[3] = {64, 1, (uint32_t)n_tile};
+    if (!make_map(&tm_x, c, 3, dims, strides, box)) return cuda_status(cudaErrorInvalidValue);
+  }
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaError_t e = launch_proj(false, tm_wk, tm_x, n, H, D, R, n_tile, k, st, true); e != cudaSuccess)
+    return cuda_status(e);
+  return cuda_status(launch_proj(false, tm_wv, tm_x, n, H, D, R, n_tile, v, st, true));
+}
+
+static mla_status prefill_common(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int L, int H, int D,
+                                 float scale, uint16_t *out, float *lse, int32_t *status, void *stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return MLA_ERR_ARG;
+  if (B < 1 || L < 1 || !isfinite(scale)) return MLA_ERR_ARG;
+  if (H != kHeads || D != kHeadDim) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MLA_ERR_UNSUPPORTED;
+  if ((long long)B * L * H >= (1LL << 31)) return MLA_ERR_ARG;
+  if ((L + 127) / 128 > 65535 || B > 65535) return MLA_ERR_ARG;  // grid limits
+  CUtensorMap tm_k, tm_v;
+  const uint64_t dims[3] = {(uint64_t)D, (uint64_t)H, (uint64_t)B * L};
+  const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)H * D * 2};
+  const uint32_t box[3] = {64, 1, 64};
+  if (!make_map(&tm_k, k, 3, dims, strides, box) || !make_map(&tm_v, v, 3, dims, strides, box))
+    return cuda_status(cudaErrorInvalidValue);
+  return cuda_status(launch_prefill(tm_k, tm_v, q, out, lse, B, L, scale, status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // namespace mla
 
 extern "C" {
+
+mla_status mla_prefill_expanded(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int L, int H, int D,
+                                float scale, uint16_t *out, float *lse, int32_t *status, void *stream) {
+  return mla::prefill_common(q, k, v, B, L, H, D, scale, out, lse, status, stream);
+}
+
+mla_status mla_expand_kv(const uint16_t *c, const uint16_t *w_uk, const uint16_t *w_uv, uint16_t *k, uint16_t *v,
+                         int n, int H, int D, int R, void *stream) {
+  return mla::expand_common(c, w_uk, w_uv, k, v, n, H, D, R, stream);
+}
 
 const char *mla_last_error_string(void) { return cudaGetErrorString(mla::g_last_error); }
 
@@ -235,6 +314,32 @@ mla_status mla_attend_indexed(const uint16_t *q_tilde, const uint16_t *cache, co
                               void *stream) {
   return mla::attend_common(mla::kModeIndexed, q_tilde, cache, nullptr, indices, seq_lens, B, Q, H, R, Lmax, 0, 0, 0,
                             K, scale, workspace, ws_bytes, o_latent, lse, status, stream);
+}
+
+mla_status mla_attend_up_dense(const uint16_t *q_tilde, const uint16_t *cache, const int32_t *seq_lens, int B, int Q,
+                               int H, int R, int Lmax, float scale, const uint16_t *w_uv, int D, void *workspace,
+                               size_t ws_bytes, uint16_t *out, uint16_t *o_latent, float *lse, int32_t *status,
+                               void *stream) {
+  return mla::attend_common(mla::kModeDense, q_tilde, cache, nullptr, nullptr, seq_lens, B, Q, H, R, Lmax, 0, 0, 0,
+                            0, scale, workspace, ws_bytes, o_latent, lse, status, stream, w_uv, D, out);
+}
+
+mla_status mla_attend_up_paged(const uint16_t *q_tilde, const uint16_t *pool, const int32_t *page_table,
+                               const int32_t *seq_lens, int B, int Q, int H, int R, int page_size, int max_pages,
+                               int num_pages, float scale, const uint16_t *w_uv, int D, void *workspace,
+                               size_t ws_bytes, uint16_t *out, uint16_t *o_latent, float *lse, int32_t *status,
+                               void *stream) {
+  return mla::attend_common(mla::kModePaged, q_tilde, pool, page_table, nullptr, seq_lens, B, Q, H, R, 0, page_size,
+                            max_pages, num_pages, 0, scale, workspace, ws_bytes, o_latent, lse, status, stream, w_uv,
+                            D, out);
+}
+
+mla_status mla_attend_up_indexed(const uint16_t *q_tilde, const uint16_t *cache, const int32_t *indices,
+                                 const int32_t *seq_lens, int B, int Q, int H, int R, int Lmax, int K, float scale,
+                                 const uint16_t *w_uv, int D, void *workspace, size_t ws_bytes, uint16_t *out,
+                                 uint16_t *o_latent, float *lse, int32_t *status, void *stream) {
+  return mla::attend_common(mla::kModeIndexed, q_tilde, cache, nullptr, indices, seq_lens, B, Q, H, R, Lmax, 0, 0, 0,
+                            K, scale, workspace, ws_bytes, o_latent, lse, status, stream, w_uv, D, out);
 }
 
 size_t mla_attend_workspace_bytes(int B, int Q, int H, int R) {

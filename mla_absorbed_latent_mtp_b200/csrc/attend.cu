@@ -29,6 +29,7 @@
 
 #include "internal.h"
 #include "sm100.cuh"
+#include "split.cuh"
 
 namespace mla {
 namespace attend {
@@ -81,9 +82,8 @@ __device__ __forceinline__ int seq_rows(const AttendParams &p, int mode, int s) 
   const int cap = (mode == kModePaged) ? p.max_pages * kPageTokens : p.Lmax;
   return min(max(L, 0), cap);
 }
-__device__ __forceinline__ int num_seqs(const AttendParams &p, int mode) {
-  return mode == kModeIndexed ? p.B * p.Q : p.B;
-}
+using split::group_start;
+using split::num_seqs;
 __device__ __forceinline__ int seq_tiles(const AttendParams &p, int mode, int s) {
   return (seq_rows(p, mode, s) + kTile - 1) / kTile;
 }
@@ -97,8 +97,6 @@ __device__ long long warp_total_tiles(const AttendParams &p, int mode, int lane)
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   return acc;
 }
-
-__device__ __forceinline__ long long group_start(long long g, long long T, long long G) { return g * T / G; }
 
 // Position of every sequence in the tile list (first tile, tile count), for the combine
 // (computed by one warp with an exclusive scan in steps of 32 sequences).
@@ -123,16 +121,21 @@ __device__ void warp_write_seq_prefix(const AttendParams &p, int mode, int lane)
 }
 
 struct Seg {
-  int s;      // sequence in the tile list
-  int lo, hi; // tile range within the sequence
-  int rows;   // data rows of the sequence
+  int s;       // sequence in the tile list
+  int lo, hi;  // tile range within the sequence (clipped to the query's causal window)
+  int rows;    // data rows of the sequence
+  bool empty;  // no tile of the range is visible to this CTA's query
 };
 
-// Walks the segments of a contiguous range [t, t_end) of the global tile list.
+// Walks the segments of a contiguous range [t, t_end) of the global tile list.  For a
+// dense or paged cache the range of query iq is clipped to the tiles holding a visible row
+// (0 .. L - Q + iq): tiles past the causal window are neither loaded nor multiplied, which
+// matters when a window holds many queries (a prefill through this path).  A segment left
+// without tiles is returned with `empty` set; its partial is written as empty.
 struct SegIter {
   long long t, t_end, base;
-  int s;
-  __device__ SegIter(long long t0, long long t1) : t(t0), t_end(t1), base(0), s(0) {}
+  int s, iq;
+  __device__ SegIter(long long t0, long long t1, int iq_) : t(t0), t_end(t1), base(0), s(0), iq(iq_) {}
   __device__ bool next(const AttendParams &p, int mode, Seg &sg) {
     if (t >= t_end) return false;
     int nt = seq_tiles(p, mode, s);
@@ -147,6 +150,13 @@ struct SegIter {
     sg.hi = (int)hi;
     sg.rows = seq_rows(p, mode, s);
     t = base + hi;
+    sg.empty = false;
+    if (mode != kModeIndexed) {
+      const int n_vis = sg.rows - p.Q + iq + 1;
+      const int vis_tiles = n_vis > 0 ? (n_vis + kTile - 1) / kTile : 0;
+      if (sg.hi > vis_tiles) sg.hi = max(vis_tiles, sg.lo);
+      sg.empty = sg.hi <= sg.lo;
+    }
     return true;
   }
 };
@@ -216,9 +226,10 @@ __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUt
                               const CUtensorMap *tm_qt, int iq, long long t0, long long t1, int lane) {
   uint64_t *bar = sh.bar;
   uint32_t tile_k = 0, q_use = 0;
-  SegIter it(t0, t1);
+  SegIter it(t0, t1, iq);
   Seg sg;
   while (it.next(p, kMode, sg)) {
+    if (sg.empty) continue;
     const int b = (kMode == kModeIndexed) ? sg.s / p.Q : sg.s;
     const int qi = (kMode == kModeIndexed) ? sg.s % p.Q : iq;
     const int qrow0 = (b * p.Q + qi) * kRows;
@@ -335,16 +346,17 @@ __device__ __forceinline__ void prepare_slot(uint32_t sbase, int n_valid, int la
 // touch disjoint TMEM columns, so the pipe simply interleaves them.  Loop state and MMA
 // operands are warp-uniform; one elected lane issues.
 template <int kMode>
-__device__ void score_mma_role(const AttendParams &p, const Shared &sh, uint32_t tmem, long long t0, long long t1,
-                               int lane) {
+__device__ void score_mma_role(const AttendParams &p, const Shared &sh, uint32_t tmem, int iq, long long t0,
+                               long long t1, int lane) {
   uint64_t *bar = sh.bar;
   constexpr uint32_t idesc_s = idesc_bf16_f32(kTile, kRows, false, false);
   const uint32_t c_base = smem_u32(sh.slot(0));
   const uint32_t qt_base = smem_u32(sh.qt(0));
   uint32_t ns = 0, q_use = 0;
-  SegIter it(t0, t1);
+  SegIter it(t0, t1, iq);
   Seg sg;
   while (it.next(p, kMode, sg)) {
+    if (sg.empty) continue;
     if (!wait_warp(&bar[kBarQFull], q_use & 1, sh, p.status)) return;
     ++q_use;
     for (int t = sg.lo; t < sg.hi; ++t, ++ns) {
@@ -383,15 +395,17 @@ __device__ void score_mma_role(const AttendParams &p, const Shared &sh, uint32_t
 }
 
 template <int kMode>
-__device__ void value_mma_role(const AttendParams &p, const Shared &sh, uint32_t tmem, long long t0, long long t1) {
+__device__ void value_mma_role(const AttendParams &p, const Shared &sh, uint32_t tmem, int iq, long long t0,
+                               long long t1) {
   uint64_t *bar = sh.bar;
   constexpr uint32_t idesc_o = idesc_bf16_f32(128, kRows, true, true);
   const uint32_t c_base = smem_u32(sh.slot(0));
   const uint32_t p_base = smem_u32(sh.pbuf(0));
   uint32_t no = 0, o_use = 0;
-  SegIter it(t0, t1);
+  SegIter it(t0, t1, iq);
   Seg sg;
   while (it.next(p, kMode, sg)) {
+    if (sg.empty) continue;
     if (!wait_warp(&bar[kBarOEmpty], (o_use & 1) ^ 1, sh, p.status)) return;
     for (int t = sg.lo; t < sg.hi; ++t, ++no) {
       if (!wait_warp(&bar[kBarPFull + (no & 1)], (no >> 1) & 1, sh, p.status)) return;
@@ -456,9 +470,18 @@ __device__ void softmax_role(const AttendParams &p, const Shared &sh, uint32_t t
   uint32_t n = 0, o_use = 0;    // tiles seen by this CTA, segments finished
   if (tid < 32) m_used[col0 + tid] = -INFINITY;
   named_bar_sync(bar_id, 128);
-  SegIter it(t0, t1);
+  SegIter it(t0, t1, iq);
   Seg sg;
   while (it.next(p, kMode, sg)) {
+    if (sg.empty) {
+      // no visible tile: an empty partial (weight zero in the merge)
+      if (tid < 32) {
+        const long long slot = split::partial_slot(p, kMode, g, sg.s, iq);
+        p.part_m[slot * kRows + col0 + tid] = -INFINITY;
+        p.part_l[slot * kRows + col0 + tid] = 0.f;
+      }
+      continue;
+    }
     const int qi = (kMode == kModeIndexed) ? sg.s % p.Q : iq;
     // positions of this CTA's query that are visible: dense/paged rows 0..L_b-Q+qi, or the list
     const int n_vis = (kMode == kModeIndexed) ? p.K : sg.rows - p.Q + qi + 1;
@@ -611,8 +634,7 @@ __device__ void softmax_role(const AttendParams &p, const Shared &sh, uint32_t t
       }
     named_bar_sync(bar_id, 128);
     if (*sh.abort_flag) return;
-    const long long slot =
-        (kMode == kModeIndexed) ? (long long)g + sg.s : ((long long)g + sg.s) * p.Q + iq;
+    const long long slot = split::partial_slot(p, kMode, g, sg.s, iq);
     if (tid < 32) {
       const int c = col0 + tid;
       p.part_m[slot * kRows + c] = m_used[c];
@@ -701,9 +723,9 @@ __global__ void __launch_bounds__(384, 1)
     }
     if (kMode == kModeIndexed || lane == 0) producer_role<kMode>(p, sh, &tm_cache, &tm_qt, iq, t0, t1, lane);
   } else if (warp == 1) {
-    score_mma_role<kMode>(p, sh, tmem, t0, t1, lane);
+    score_mma_role<kMode>(p, sh, tmem, iq, t0, t1, lane);
   } else if (warp == 10) {
-    value_mma_role<kMode>(p, sh, tmem, t0, t1);
+    value_mma_role<kMode>(p, sh, tmem, iq, t0, t1);
   } else {
     softmax_role<kMode>(p, sh, tmem, g, iq, t0, t1, warp, lane);
   }
@@ -752,18 +774,10 @@ __global__ void __launch_bounds__(128, 4) combine_kernel(const AttendParams p, i
   __shared__ long long sh_T, sh_g_first;
   __shared__ int sh_nslot;
   if (tid == 0) {
-    const int ns = num_seqs(p, mode);
-    const long long T = p.seq_ts[ns - 1] + p.seq_nt[ns - 1];
-    const long long ts = p.seq_ts[s];
-    const int nt = p.seq_nt[s];
-    long long g_first = 0, g_last = -1;
-    if (nt > 0) {
-      g_first = ((ts + 1) * G - 1) / T;
-      g_last = ((ts + nt) * G - 1) / T;
-    }
-    sh_T = T;
-    sh_g_first = g_first;
-    sh_nslot = (int)(g_last - g_first + 1);
+    const split::GroupRange gr = split::seq_group_range(p, mode, s);
+    sh_T = gr.T;
+    sh_g_first = gr.g_first;
+    sh_nslot = gr.nslot;
     if (blockIdx.y == 0 && i == 0 && mode != kModeIndexed && p.seq_lens != nullptr) {
       const int L = p.seq_lens[b];
       const int cap = (mode == kModePaged) ? p.max_pages * kPageTokens : p.Lmax;
@@ -790,8 +804,8 @@ __global__ void __launch_bounds__(128, 4) combine_kernel(const AttendParams p, i
 #pragma unroll
     for (int j = 0; j < kCombineChunk; ++j) {
       const long long gg = g_first + k0 + j;
-      const bool live = (k0 + j < nslot) && (all_live || group_start(gg, T, G) < group_start(gg + 1, T, G));
-      const long long slot = (mode == kModeIndexed) ? gg + s : (gg + s) * p.Q + i;
+      const bool live = (k0 + j < nslot) && (all_live || split::group_live(gg, T, G));
+      const long long slot = split::partial_slot(p, mode, gg, s, i);
 #pragma unroll
       for (int hh = 0; hh < kCombineHeads; ++hh) {
         const long long row = slot * kRows + h0 + hh;
@@ -816,6 +830,7 @@ __global__ void __launch_bounds__(128, 4) combine_kernel(const AttendParams p, i
 #pragma unroll
       for (int j = 0; j < kCombineChunk; ++j) {
         const float w = exp2f(mk[hh][j] - mx);  // 0 for empty slots (m = -inf)
+        if (w == 0.f) continue;                  // an empty partial's O is never summed in
         den[hh] += w * lk[hh][j];
         acc[hh].x += w * ok[hh][j].x;
         acc[hh].y += w * ok[hh][j].y;
@@ -904,7 +919,7 @@ size_t attend_workspace_bytes_for(int B, int Q, int sms) {
 
 template <int kMode>
 static cudaError_t launch_attend_mode(const CUtensorMap &tm_cache, const CUtensorMap &tm_qt, const AttendParams &p,
-                                      cudaStream_t stream) {
+                                      cudaStream_t stream, bool with_combine) {
   static int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -917,20 +932,20 @@ static cudaError_t launch_attend_mode(const CUtensorMap &tm_cache, const CUtenso
   const int grid = p.groups * p.group_size;
   cudaError_t e = launch_chained(attend::attend_kernel<kMode>, dim3(grid), dim3(attend::kThreads), attend::kSmemBytes,
                                  stream, tm_cache, tm_qt, p);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || !with_combine) return e;
   dim3 cgrid(p.B * p.Q, kHeads / attend::kCombineHeads);
   return launch_chained(attend::combine_kernel, cgrid, dim3(128), 0, stream, p, (int)kMode);
 }
 
 cudaError_t launch_attend(int mode, const CUtensorMap &tm_cache, const CUtensorMap &tm_qt, const AttendParams &p,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, bool with_combine) {
   switch (mode) {
     case kModeDense:
-      return launch_attend_mode<kModeDense>(tm_cache, tm_qt, p, stream);
+      return launch_attend_mode<kModeDense>(tm_cache, tm_qt, p, stream, with_combine);
     case kModePaged:
-      return launch_attend_mode<kModePaged>(tm_cache, tm_qt, p, stream);
+      return launch_attend_mode<kModePaged>(tm_cache, tm_qt, p, stream, with_combine);
     default:
-      return launch_attend_mode<kModeIndexed>(tm_cache, tm_qt, p, stream);
+      return launch_attend_mode<kModeIndexed>(tm_cache, tm_qt, p, stream, with_combine);
   }
 }
 

@@ -43,8 +43,13 @@ struct AttendParams {
 size_t attend_slots(int B, int Q, int sms);
 size_t attend_workspace_bytes_for(int B, int Q, int sms);
 
+// The attend kernel, then (with_combine) the split-L combine that writes o_latent / lse.
 cudaError_t launch_attend(int mode, const CUtensorMap &tm_cache, const CUtensorMap &tm_qt,
-                          const AttendParams &p, cudaStream_t stream);
+                          const AttendParams &p, cudaStream_t stream, bool with_combine = true);
+// The split-L merge fused with the W_UV up-projection: out [B*Q, H, D] from the attend
+// kernel's partials (o_latent / lse in p written too when non-null).
+cudaError_t launch_merge_up(const CUtensorMap &tm_w, const AttendParams &p, int mode, uint16_t *out,
+                            cudaStream_t stream);
 cudaError_t launch_debug_gather(int mode, const uint16_t *src, const int32_t *page_table,
                                 const int32_t *indices, int B, int Q, int R, int Lmax, int max_pages,
                                 int num_pages, int K, const int32_t *req, int n_req, uint16_t *out,
@@ -53,8 +58,15 @@ cudaError_t launch_debug_gather(int mode, const uint16_t *src, const int32_t *pa
 // Per-head projection GEMM: out[n, h, m] = sum_k A_h[m, k] * X[n, h, k].
 // absorb (a_mn_major = true):  A_h[m=r, k=d] = W_UK[h][d][r]  (M = R, K = D)
 // up-proj (a_mn_major = false): A_h[m=d, k=r] = W_UV[h][d][r] (M = D, K = R)
+// x_bcast: X is [n, K] (one row per token for every head), read with head coordinate 0.
 cudaError_t launch_proj(bool a_mn_major, const CUtensorMap &tm_w, const CUtensorMap &tm_x, int n, int H,
-                        int M_total, int K_total, int n_tile, uint16_t *out, cudaStream_t stream);
+                        int M_total, int K_total, int n_tile, uint16_t *out, cudaStream_t stream,
+                        bool x_bcast = false);
+
+// Causal self-attention of B sequences of L tokens in the expanded form (64 heads of 256):
+// q, out [B, L, H, D]; k, v through tensor maps over [B*L, H, D] (boxes of 64 dims x 64 tokens).
+cudaError_t launch_prefill(const CUtensorMap &tm_k, const CUtensorMap &tm_v, const uint16_t *q, uint16_t *out,
+                           float *lse, int B, int L, float scale, int32_t *status, cudaStream_t stream);
 
 int device_sm_count();
 cudaError_t launch_wait_timeout(long long limit_cycles, int32_t *status, cudaStream_t stream);

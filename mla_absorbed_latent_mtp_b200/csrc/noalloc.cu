@@ -12,8 +12,10 @@
 namespace {
 
 // 32 MiB of scratch: enough for mla_attend_workspace_bytes(B, Q, 64, 512) up to 32 MiB
-// (for example B * Q up to about 100 on a 148-SM device).  Every GPU that loads the library
-// holds this array until the process exits.
+// (for example B * Q up to about 100 on a 148-SM device).  The runtime reserves it on a
+// device when it loads this file's code module there: with lazy module loading (the
+// default), at the first cudaGetSymbolAddress below, i.e. the first call on that device.
+// It is held until the process exits.
 constexpr size_t kScratchBytes = size_t(32) << 20;
 __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 

@@ -31,6 +31,7 @@ __host__ __device__ constexpr int smem_bytes(int stages, int n_tile) {
 
 struct Params {
   int n, H, M_total, K_total, n_tile, stages;
+  int x_bcast;  // 1: X has one row per token shared by every head (X[n][k], the latents c)
   uint16_t *out;
 };
 
@@ -96,13 +97,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         load_a(kc, kc);
       }
       grid_dep_wait();
-      for (int kc = 0; kc < pre; ++kc) tma_load_3d(b_stage0 + kc * b_bytes, &tm_x, &full[kc], kc * kBK, h, nt * NT);
+      const int xh = p.x_bcast ? 0 : h;
+      for (int kc = 0; kc < pre; ++kc) tma_load_3d(b_stage0 + kc * b_bytes, &tm_x, &full[kc], kc * kBK, xh, nt * NT);
       for (int kc = pre; kc < nk; ++kc) {
         const int s = kc % kStages, use = kc / kStages;
         if (!mbar_wait(&empty[s], (use & 1) ^ 1, abort_flag, nullptr)) break;
         mbar_arrive_expect_tx(&full[s], kABytes + NT * kBK * 2);
         load_a(kc, s);
-        tma_load_3d(b_stage0 + s * b_bytes, &tm_x, &full[s], kc * kBK, h, nt * NT);
+        tma_load_3d(b_stage0 + s * b_bytes, &tm_x, &full[s], kc * kBK, xh, nt * NT);
       }
     }
   } else if (warp == 1) {
@@ -178,11 +180,11 @@ static cudaError_t launch_proj_t(const CUtensorMap &tm_w, const CUtensorMap &tm_
 }
 
 cudaError_t launch_proj(bool a_mn_major, const CUtensorMap &tm_w, const CUtensorMap &tm_x, int n, int H,
-                        int M_total, int K_total, int n_tile, uint16_t *out, cudaStream_t stream) {
+                        int M_total, int K_total, int n_tile, uint16_t *out, cudaStream_t stream, bool x_bcast) {
   // keep every K chunk of the weight block in flight when it fits
   int stages = std::min(proj::kMaxStages, K_total / proj::kBK);
   while (stages > 2 && proj::smem_bytes(stages, n_tile) > proj::kSmemLimit) --stages;
-  proj::Params p{n, H, M_total, K_total, n_tile, stages, out};
+  proj::Params p{n, H, M_total, K_total, n_tile, stages, x_bcast ? 1 : 0, out};
   return a_mn_major ? launch_proj_t<true>(tm_w, tm_x, p, stream) : launch_proj_t<false>(tm_w, tm_x, p, stream);
 }
 

@@ -75,3 +75,15 @@ def test_recorded_traffic_is_close_to_the_algorithmic_bytes():
     for (name, _src), traffic in bench.TRAFFIC.items():
         cache = bench.step_bytes(synth.make_workload(name, with_data=False))["cache"]
         assert cache <= traffic <= 1.1 * cache, (name, traffic, cache)
+
+
+@pytest.mark.parametrize("L", [1, 5, 64, 130])
+def test_prefill_flop_counts(L):
+    """A prefill's causal (query, key) pairs, counted one by one; the absorbed attention does
+    twice the expanded one's arithmetic per pair (512-wide latent against 256-wide heads)."""
+    pairs = sum(1 for t in range(L) for j in range(L) if j <= t)
+    f = bench.prefill_flops(L)
+    assert f["expanded_attention"] == pairs * 64 * 2 * 2 * 256
+    assert f["absorbed_attention"] == 2 * f["expanded_attention"]
+    assert f["expanded"] - f["expanded_attention"] == 2 * 2 * L * 512 * 64 * 256
+    assert f["absorbed"] - f["absorbed_attention"] == 2 * 2 * L * 64 * 256 * 512

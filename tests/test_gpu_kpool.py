@@ -45,10 +45,21 @@ def _check_lists(got, pooled_ref, wq, lens, Q, pool, topk, with_tail):
             g = got[b, i]
             if np.array_equal(g, ref):
                 continue
-            # only near-ties may differ: same layout, and the swapped pools' scores agree
+            # Several lists are correct when pools tie; whatever the GPU chose must still be a
+            # valid list: whole, complete, visible pools in ascending order, then -1 up to topk,
+            # then the same tail.  Only near-ties may be swapped.
             n_sel = max(pos + 1, 0) // pool
+            head = [int(x) for x in g[:topk]]
+            used = [x for x in head if x >= 0]
+            assert head == used + [-1] * (topk - len(used)), (b, i, "padding must follow the pools")
+            assert len(used) % pool == 0, (b, i)
+            chosen = [used[k] // pool for k in range(0, len(used), pool)]
+            for k, p in enumerate(chosen):
+                assert used[k * pool:(k + 1) * pool] == list(range(p * pool, (p + 1) * pool)), (b, i, p)
+            assert chosen == sorted(set(chosen)), (b, i, "pools ascending and distinct")
+            assert all(0 <= p < n_sel for p in chosen), (b, i, "only complete, visible pools")
             scores = pooled_ref[b][:n_sel] @ w
-            gs = {int(x) // pool for x in g[:topk] if x >= 0}
+            gs = set(chosen)
             rs = {int(x) // pool for x in ref[:topk] if x >= 0}
             assert len(gs) == len(rs)
             kth = min(scores[p] for p in rs)

@@ -60,3 +60,31 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     with pytest.raises(m.MLAError) as e:
         m.mla_attend_dense_noalloc(qt, cache)
     assert e.value.code == m.MLA_ERR_WORKSPACE
+
+
+def test_noalloc_call_allocates_no_device_memory_and_runs_on_a_side_stream():
+    """The point of the entry point: with its outputs supplied, a call takes no device memory
+    (the free-memory figure of the device does not move), and on a side stream it gives the
+    same result once that stream is synchronised."""
+    wl = tiny_workload("dense", 2, 6, [900, 300], H=64, D=256, R=512, seed=33)
+    qt = to_dev(synthetic_qtilde(2, 6, seed=3))
+    cache, lens = to_dev(wl.cache), ints_to_dev(wl.seq_lens)
+    o = torch.empty(2, 6, 64, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(2, 6, 64, dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    m.mla_attend_dense_noalloc(qt, cache, lens, wl.scale, o_latent=o, lse=lse, status=st)  # first call: set-up
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    m.mla_attend_dense_noalloc(qt, cache, lens, wl.scale, o_latent=o, lse=lse, status=st)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    ref = o.clone()
+    side = torch.cuda.Stream()
+    o2 = torch.zeros_like(o)
+    lse2 = torch.zeros_like(lse)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        m.mla_attend_dense_noalloc(qt, cache, lens, wl.scale, o_latent=o2, lse=lse2, status=st, stream=side)
+    side.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(o2, ref)
