@@ -457,6 +457,27 @@ HEADLINE = "ragged_paged_decode"
 E2E_BYTES_CAP = 24e9
 
 
+def steps_per_graph(K, n_rot=1, cap=32):
+    """Steps captured per CUDA graph: the largest divisor of K up to `cap`, preferring a
+    multiple of the number of index-list sets the steps rotate through."""
+    divisors = [g for g in range(1, min(K, cap) + 1) if K % g == 0]
+    rot = [g for g in divisors if g % n_rot == 0]
+    return max(rot) if rot else max(divisors)
+
+
+def capture(fn, n, idx_turn=None):
+    """A CUDA graph of n calls of fn (the library's launches go to torch's capture stream).
+    The index-list rotation restarts at the first set in every graph."""
+    import torch
+    if idx_turn is not None:
+        idx_turn[0] = 0
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(n):
+            fn()
+    return g
+
+
 def _seq_len(name, args):
     """Rows per sequence for a profiling-size run (MTP verify: prefix + the 6 window rows)."""
     if args.seq_len is None:
@@ -525,40 +546,7 @@ def measure_config(name, args, device, rank, world, clocks, peaks, peak_kind, sr
     def up():
         m.mla_up_proj(o, w_uv, out)
 
-    for _ in range(args.warmup):
-        absorb(); attend(); up()
-    torch.cuda.synchronize()
-    assert int(status.item()) == 0, m.status_string(int(status.item()))
-
-    K = args.steps
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    wall0 = time.time()
-    # the timed steps: nothing between the launches, so each kernel may start while the
-    # previous one drains (the library chains its launches)
-    start.record()
-    for k in range(K):
-        absorb(); attend(); up()
-    stop.record()
-    torch.cuda.synchronize()
-    wall1 = time.time()
-    barrier()
-    local_ms = start.elapsed_time(stop) / K
-    ms, value = aggregate(local_ms, acc["total"], device)
-    # per-stage breakdown in a separate pass: events between the stages serialise them
-    Kb = max(1, min(K, 50))
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(Kb)]
-    torch.cuda.synchronize()
-    for k in range(Kb):
-        e = ev[k]
-        e[0].record(); absorb(); e[1].record(); attend(); e[2].record(); up(); e[3].record()
-    torch.cuda.synchronize()
-    stage = [sum(ev[k][j].elapsed_time(ev[k][j + 1]) for k in range(Kb)) / Kb for j in range(3)]
-    stage = reduce_max(stage, device)
-    launches = K * 4  # absorb, attend, split-L combine, up-projection
-    # the same step with the up-projection fused into the split-L merge (mla_attend_up_*):
-    # absorb, attend, merge + up-projection
+    # the fused path: the up-projection runs inside the split-L merge (mla_attend_up_*)
     def attend_up():
         if wl.mode == "dense":
             m.mla_attend_up_dense(qt, cache, w_uv, lens, wl.scale, ws, out, None, lse, status)
@@ -569,46 +557,86 @@ def measure_config(name, args, device, rank, world, clocks, peaks, peak_kind, sr
                                     None, lse, status)
             idx_turn[0] += 1
 
-    for _ in range(args.warmup):
+    def chained_step():
+        absorb(); attend(); up()
+
+    def fused_step():
         absorb(); attend_up()
+
+    for _ in range(args.warmup):
+        chained_step()
+        fused_step()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, m.status_string(int(status.item()))
+
+    # Every timed loop replays CUDA graphs: the host-side cost of a launch through Python
+    # (tens of microseconds) would otherwise set the pace of the short workloads.  A graph
+    # holds G steps (for the index-list workload a multiple of the list sets it cycles
+    # through); the loops replay K / G of them, so exactly K steps run.
+    K = args.steps
+    G = steps_per_graph(K, len(idx_sets))
+    g_chained = capture(chained_step, G, idx_turn)
+    g_fused = capture(fused_step, G, idx_turn)
+    for _ in range(max(1, -(-args.warmup // G))):
+        g_chained.replay()
+        g_fused.replay()
+    torch.cuda.synchronize()
+
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    # the timed steps: nothing between the launches, so each kernel may start while the
+    # previous one drains (the library chains its launches)
+    start.record()
+    for _ in range(K // G):
+        g_chained.replay()
+    stop.record()
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    barrier()
+    local_ms = start.elapsed_time(stop) / K
+    ms, value = aggregate(local_ms, acc["total"], device)
+
     f_start, f_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
+    fw0 = time.time()
     f_start.record()
-    for _ in range(K):
-        absorb(); attend_up()
+    for _ in range(K // G):
+        g_fused.replay()
     f_stop.record()
     torch.cuda.synchronize()
+    fw1 = time.time()
+    barrier()
     fused_ms, fused_value = aggregate(f_start.elapsed_time(f_stop) / K, acc["total"], device)
-    # the attend kernel and the fused merge + up-projection alone, back to back
-    Kf = max(20, min(K, 400))
-    k_start, k_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    k_start.record()
-    for _ in range(Kf):
-        attend_up()
-    k_stop.record()
-    torch.cuda.synchronize()
-    attend_up_ms = reduce_max([k_start.elapsed_time(k_stop) / Kf], device)[0]
     # the step the line reports: whichever path (chained or fused) is faster on this workload
     best = "fused" if fused_ms < ms else "chained"
-    if best == "fused":
-        launches = K * 3  # absorb, attend, merge + up-projection
-    # the attend + combine launches alone, back to back on the same stream: the duration
-    # of the pair as it runs inside the step (chained, nothing serialising it), for the
-    # roofline; the per-stage pass above puts events between the stages, which serialises
-    # every launch and adds its start-up to the stage
-    Ka = max(20, min(K, 400))
-    a_start, a_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
+    launches = K * (3 if best == "fused" else 4)
+
+    # Each stage alone, Kb times back to back in one graph (stage time = graph time / Kb),
+    # and the attend call (attend + split-L combine) the same way: its duration as it runs
+    # inside the step, for the roofline.  The fused attend (attend + merge + up-projection)
+    # likewise.
+    Kb = max(len(idx_sets), min(K, 50) // len(idx_sets) * len(idx_sets))
+
+    def timed_graph(fn, reps):
+        g = capture(fn, reps, idx_turn)
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    stage = reduce_max([timed_graph(absorb, Kb), timed_graph(attend, Kb), timed_graph(up, Kb)], device)
     aw0 = time.time()
-    a_start.record()
-    for _ in range(Ka):
-        attend()
-    a_stop.record()
-    torch.cuda.synchronize()
+    att_ms = reduce_max([timed_graph(attend, max(Kb, 20))], device)[0]
     aw1 = time.time()
-    att_ms = reduce_max([a_start.elapsed_time(a_stop) / Ka], device)[0]
+    attend_up_ms = reduce_max([timed_graph(attend_up, max(Kb, 20))], device)[0]
+    del g_chained, g_fused
 
     # end to end through the public API with host buffers: H2D inputs, D2H output per step
     h2d = host_cache.numel() * 2 + host_q.numel() * 2 + host_lens.numel() * 4
@@ -651,8 +679,12 @@ def measure_config(name, args, device, rank, world, clocks, peaks, peak_kind, sr
         "e2e": {"value": e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e_ms, "steps": Ke},
         "gpu_launches": launches,
-        "clocks": clocks.summary(wall0, wall1),
+        "roofline_fused": dict(attend_roofline(acc, attend_up_ms, peaks, peak_kind, None),
+                               kernel="attend_kernel + merge_up_kernel (mla_attend_up_*: attend, split-L merge "
+                                      "and W_UV up-projection)"),
+        "clocks": clocks.summary(wall0, wall1) if best == "chained" else clocks.summary(fw0, fw1),
         "clocks_attend_chained": clocks.summary(aw0, aw1),
+        "timing": f"device time (CUDA events) around replays of CUDA graphs of {G} steps",
     }
     if cpu_seconds > 0:
         if wl.mode == "indexed":

@@ -59,7 +59,7 @@ constexpr int kOffBar = kOffAlpha + 64 * 4;
 constexpr int kBarCFull = 0, kBarCEmpty = kSlots, kBarQFull = 2 * kSlots, kBarQEmpty = kBarQFull + 1,
               kBarSFull = kBarQEmpty + 1, kBarSEmpty = kBarSFull + 2, kBarPFull = kBarSEmpty + 2,
               kBarPEmpty = kBarPFull + 2, kBarOFull = kBarPEmpty + 2, kBarOEmpty = kBarOFull + 1,
-              kNumBars = kBarOEmpty + 1;
+              kBarDrain = kBarOEmpty + 1, kNumBars = kBarDrain + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemUsed = kOffMisc + 16;
 constexpr int kSmemBytes = kSmemUsed + 1024;  // slack for 1024-byte alignment of the base
@@ -221,11 +221,13 @@ __device__ __forceinline__ uint32_t ring_pos(uint32_t k) { return k % kSlots; }
 __device__ __forceinline__ uint32_t ring_use(uint32_t k) { return k / kSlots; }
 
 // ------------------------------------------------------------------ producer (warp 0)
+// Issues the loads; counts the q~ loads and the ring-slot loads it issued (for the drain).
 template <int kMode>
-__device__ void producer_role(const AttendParams &p, const Shared &sh, const CUtensorMap *tm_cache,
-                              const CUtensorMap *tm_qt, int iq, long long t0, long long t1, int lane) {
+__device__ void producer_loads(const AttendParams &p, const Shared &sh, const CUtensorMap *tm_cache,
+                               const CUtensorMap *tm_qt, int iq, long long t0, long long t1, int lane,
+                               uint32_t &q_use, uint32_t &slots_issued) {
   uint64_t *bar = sh.bar;
-  uint32_t tile_k = 0, q_use = 0;
+  uint32_t tile_k = 0;
   SegIter it(t0, t1, iq);
   Seg sg;
   while (it.next(p, kMode, sg)) {
@@ -268,8 +270,8 @@ __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUt
             if (k < p.K) nxt[m] = list[k];
           }
         }
-        const uint16_t *src[2];
-        uint32_t nbytes[2];
+        // cache row (in units of R) of the tile rows lane and lane + 32, -1 when unused
+        int rowi[2];
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
           const int k = t * kTile + lane + 32 * m;
@@ -278,26 +280,27 @@ __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUt
           const bool used = k < p.K && cur[m] != kUnusedEntry;
           if (used) row = indexed_row_of(b, cur[m], p.Lmax, limit, bad);
           if (bad) report_status(p.status, kStatusIndex);
-          src[m] = p.cache + row * kLatent;
-          nbytes[m] = (used && !bad) ? 16u : 0u;
+          rowi[m] = (used && !bad) ? (int)row : -1;
         }
+        // Each copy instruction moves two tile rows' 256-byte slice of this slot: lanes
+        // 0-15 row 2i, lanes 16-31 row 2i + 1, 16 bytes each, so every instruction reads four
+        // whole 128-byte lines (B * Lmax < 2^31 rows, so a row fits an int).
+        const int u = lane & 15, at = u >> 3, pc = u & 7;
         for (int qq = 0; qq < kSlotQuarters; ++qq) {
           const uint32_t k = tile_k * kSlotQuarters + qq;
           const uint32_t rp = ring_pos(k);
           if (!wait_warp(&bar[kBarCEmpty + rp], (ring_use(k) & 1) ^ 1, sh, p.status)) return;
-          const uint32_t dst_s = smem_u32(sh.slot(rp));
+          const uint32_t dst_s = smem_u32(sh.slot(rp)) + at * kAtomBytes;
+          const uint16_t *src_q = p.cache + qq * 128 + at * 64 + pc * 8;
 #pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            const int r = lane + 32 * m;
-#pragma unroll
-            for (int at = 0; at < 2; ++at) {
-              const uint32_t dst_r = dst_s + at * kAtomBytes + r * 128;
-#pragma unroll
-              for (int pc = 0; pc < 8; ++pc)
-                cp_async_16(dst_r + ((pc ^ (r & 7)) << 4), src[m] + qq * 128 + at * 64 + pc * 8, nbytes[m]);
-            }
+          for (int i = 0; i < kTile / 2; ++i) {
+            const int r = 2 * i + (lane >> 4);
+            const int ri = __shfl_sync(0xffffffffu, rowi[i >> 4], r & 31);
+            cp_async_16(dst_s + r * 128 + ((pc ^ (r & 7)) << 4), src_q + (long long)max(ri, 0) * kLatent,
+                        ri >= 0 ? 16u : 0u);
           }
           cp_async_arrive_noinc(&bar[kBarCFull + rp]);
+          slots_issued = k + 1;
         }
       } else {
         const int j0 = t * kTile;
@@ -316,9 +319,25 @@ __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUt
           mbar_arrive_expect_tx(&bar[kBarCFull + rp], kSlotBytes);
           tma_load_2d(sh.slot(rp), tm_cache, &bar[kBarCFull + rp], qq * 128, (int)row);
           tma_load_2d(sh.slot(rp) + kAtomBytes, tm_cache, &bar[kBarCFull + rp], qq * 128 + 64, (int)row);
+          slots_issued = k + 1;
         }
       }
     }
+  }
+}
+
+// The producer role: the loads, then (also after an abort) a wait until every copy it
+// issued has landed.
+template <int kMode>
+__device__ void producer_role(const AttendParams &p, const Shared &sh, const CUtensorMap *tm_cache,
+                              const CUtensorMap *tm_qt, int iq, long long t0, long long t1, int lane) {
+  uint32_t q_use = 0, slots_issued = 0;
+  producer_loads<kMode>(p, sh, tm_cache, tm_qt, iq, t0, t1, lane, q_use, slots_issued);
+  if constexpr (kMode == kModeIndexed) cp_async_wait_all();  // this lane's row copies
+  if (lane == 0) {
+    bool ok = drain_ring(&sh.bar[kBarQFull], 1, q_use);
+    if constexpr (kMode != kModeIndexed) ok = drain_ring(&sh.bar[kBarCFull], kSlots, slots_issued) && ok;
+    if (!ok) report_status(p.status, kStatusTimeout);
   }
 }
 
@@ -697,6 +716,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(&sh.bar[kBarOFull], 1);
     mbar_init(&sh.bar[kBarOEmpty], kSoftmaxWarps);
+    mbar_init(&sh.bar[kBarDrain], 2);
     *sh.abort_flag = 0;
     fence_barrier_init();
   }
@@ -731,17 +751,20 @@ __global__ void __launch_bounds__(384, 1)
   }
 
   __syncwarp();
+  // After an abort, the MMAs issued by the two MMA warps (lane 0 of each) must finish
+  // before TMEM is released: each commits to the drain barrier, warp 1 waits for both.
+  // (The producer has already waited for its copies.)
+  if (warp == 10 && *sh.abort_flag) {
+    if (lane == 0) umma_commit(&sh.bar[kBarDrain]);
+    __syncwarp();
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     if (*sh.abort_flag) {
-      // drain: let every issued MMA finish before TMEM is released, and give in-flight
-      // copies time to land before the shared memory is handed to another CTA
       if (lane == 0) {
-        umma_commit(&sh.bar[kBarOFull]);
-        const long long t_start = clock64();
-        while (clock64() - t_start < 2000000) {
-        }
+        umma_commit(&sh.bar[kBarDrain]);
+        if (!mbar_wait_drain(&sh.bar[kBarDrain], 0)) report_status(p.status, kStatusTimeout);
       }
       __syncwarp();
     }

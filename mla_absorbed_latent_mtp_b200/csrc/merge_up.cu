@@ -41,12 +41,14 @@ constexpr int kStageBytes = kNTile * kHeadDim * 4;  // fp32 D staged as [row][d]
 constexpr int kOffW = 0;
 constexpr int kOffB = kOffW + kWBytes;
 constexpr int kOffStage = kOffB + kBBytes;
-constexpr int kOffBar = kOffStage + kStageBytes;
+constexpr int kOffRows = kOffStage + kStageBytes;        // RowInfo per query row of the tile
+constexpr int kOffBar = kOffRows + kNTile * 32;
 constexpr int kOffMisc = kOffBar + 2 * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
 constexpr uint32_t kTmemCols = 2 * kNTile;
-constexpr int kMaxBatch = 8;                // partials of one row loaded together
+constexpr int kMaxBatch = 6;                // partials of each of two rows loaded together
 static_assert(kSmemBytes <= 113 * 1024, "two CTAs per SM");
+static_assert(kNTile % (2 * kWarps) == 0, "rows are merged two at a time per warp");
 static_assert(kTmemCols == 64, "TMEM allocation is a power of two >= 32");
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -60,64 +62,13 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Merges the latent chunk [r0, r0 + 128) of query row v (b = v / Q, i = v % Q) for head h.
-// Lane l returns o[r0 + 4l .. r0 + 4l + 3] (normalised; zero when the row saw nothing);
-// M and den (log2-domain max and weighted sum) come back for the log-sum-exp.
-__device__ __forceinline__ float4 merge_row(const AttendParams &p, int mode, int v, int h, int r0, int lane,
-                                            float &M, float &den) {
-  const int b = v / p.Q, i = v % p.Q;
-  const int s = (mode == kModeIndexed) ? v : b;
-  const split::GroupRange gr = split::seq_group_range(p, mode, s);
-  const long long G = p.groups;
-  M = -INFINITY;
-  for (int k = lane; k < gr.nslot; k += 32) {
-    const long long g = gr.g_first + k;
-    if (split::group_live(g, gr.T, G)) M = fmaxf(M, p.part_m[split::partial_slot(p, mode, g, s, i) * kHeads + h]);
-  }
-  M = warp_max(M);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float dsum = 0.f;
-  if (M != -INFINITY) {
-    for (int k0 = 0; k0 < gr.nslot; k0 += 32) {
-      // lane j holds the weight of partial k0 + j (0 for an empty group)
-      float w = 0.f;
-      long long my_slot = 0;
-      {
-        const int k = k0 + lane;
-        const long long g = gr.g_first + k;
-        if (k < gr.nslot && split::group_live(g, gr.T, G)) {
-          my_slot = split::partial_slot(p, mode, g, s, i);
-          w = exp2f(p.part_m[my_slot * kHeads + h] - M);
-          dsum += w * p.part_l[my_slot * kHeads + h];
-        }
-      }
-      const int cnt = min(32, gr.nslot - k0);
-      for (int j0 = 0; j0 < cnt; j0 += kMaxBatch) {
-        float4 x[kMaxBatch];
-        float wj[kMaxBatch];
-#pragma unroll
-        for (int j = 0; j < kMaxBatch; ++j) {
-          wj[j] = __shfl_sync(0xffffffffu, w, (j0 + j) & 31);
-          const long long sl = __shfl_sync(0xffffffffu, my_slot, (j0 + j) & 31);
-          x[j] = (j0 + j < cnt && wj[j] != 0.f)
-                     ? *reinterpret_cast<const float4 *>(p.part_o + (sl * kHeads + h) * kLatent + r0 + 4 * lane)
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int j = 0; j < kMaxBatch; ++j) {
-          const float a = (j0 + j < cnt) ? wj[j] : 0.f;
-          acc.x += a * x[j].x;
-          acc.y += a * x[j].y;
-          acc.z += a * x[j].z;
-          acc.w += a * x[j].w;
-        }
-      }
-    }
-  }
-  den = warp_sum(dsum);
-  const float inv = (M != -INFINITY && den > 0.f) ? 1.f / den : 0.f;
-  return make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-}
+// The split-L partials of one query row: the groups g_first .. g_first + nslot - 1 of
+// tile-list sequence s (query i) -- found once per row by one thread.
+struct RowInfo {
+  long long g_first, T;
+  int nslot, s, i, pad;
+};
+static_assert(sizeof(RowInfo) <= 32, "row table entry");
 
 __global__ void __launch_bounds__(kThreads, 2)
     merge_up_kernel(const __grid_constant__ CUtensorMap tm_w, const AttendParams p, int mode, uint16_t *out) {
@@ -160,26 +111,138 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   grid_dep_wait();  // the partials, the tile table and the lengths come from the attend kernel
 
-  // ---- merge: warp w takes query rows w, w + 8, w + 16, w + 24 of the tile
-  const uint32_t b_base = smem_u32(base + kOffB);
-  for (int t = warp; t < kNTile; t += kWarps) {
-    const int v = v0 + t;
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+  // ---- merge.  Every load of a round is issued before any is used, and the rounds are
+  // few: (1) one thread per query row finds its range of partials; (2) each warp loads the
+  // running maxima and sums of its four rows' partials (lane k: partial k) and forms the
+  // merge weights; (3) it loads the 128-wide chunk of every partial of two rows at a time
+  // (lane l: latent 4l .. 4l + 3), weighs and sums them.
+  RowInfo *rows = reinterpret_cast<RowInfo *>(base + kOffRows);
+  if (tid < kNTile) {
+    RowInfo ri = {0, 1, 0, 0, 0, 0};
+    const int v = v0 + tid;
     if (v < n) {
-      float M, den;
-      o = merge_row(p, mode, v, h, kc * kChunk, lane, M, den);
-      const uint32_t lo = pack_bf16x2(o.x, o.y), hi = pack_bf16x2(o.z, o.w);
-      if (p.o_latent != nullptr)
-        *reinterpret_cast<uint2 *>(p.o_latent + ((long long)v * kHeads + h) * kLatent + kc * kChunk + 4 * lane) =
-            make_uint2(lo, hi);
-      if (p.lse != nullptr && kc == 0 && lane == 0)
-        p.lse[(long long)v * kHeads + h] =
-            (M != -INFINITY && den > 0.f) ? (M + log2f(den)) * 0.69314718055994530942f : -INFINITY;
+      ri.i = v % p.Q;
+      ri.s = (mode == kModeIndexed) ? v : v / p.Q;
+      const split::GroupRange gr = split::seq_group_range(p, mode, ri.s);
+      ri.g_first = gr.g_first;
+      ri.T = gr.T;
+      ri.nslot = gr.nslot;
     }
-    // B operand: row t, latent 4*lane .. 4*lane+3 of the chunk, 128-byte swizzle
-    const uint32_t lo = pack_bf16x2(o.x, o.y), hi = pack_bf16x2(o.z, o.w);
-    const int atom = lane >> 4, unit = (lane & 15) >> 1;
-    st_shared_v2(b_base + atom * kBAtomBytes + t * 128 + ((unit ^ (t & 7)) << 4) + (lane & 1) * 8, lo, hi);
+    rows[tid] = ri;
+  }
+  __syncthreads();
+  const uint32_t b_base = smem_u32(base + kOffB);
+  const long long G = p.groups;
+  constexpr int kRowsPerWarp = kNTile / kWarps;  // 4
+  const RowInfo *ri = rows + warp;  // row j of this warp: ri[kWarps * j]
+  float M[kRowsPerWarp], mk[kRowsPerWarp], lk[kRowsPerWarp];
+  long long sl[kRowsPerWarp];
+  int maxslot = 0;
+#pragma unroll
+  for (int j = 0; j < kRowsPerWarp; ++j) maxslot = max(maxslot, ri[kWarps * j].nslot);
+  // (2) maxima; the first 32 partials' (m, l) stay in registers for the weights
+#pragma unroll
+  for (int j = 0; j < kRowsPerWarp; ++j) {
+    M[j] = -INFINITY;
+    mk[j] = -INFINITY;
+    lk[j] = 0.f;
+    sl[j] = 0;
+  }
+  for (int k0 = 0; k0 < maxslot; k0 += 32) {
+#pragma unroll
+    for (int j = 0; j < kRowsPerWarp; ++j) {
+      const int k = k0 + lane;
+      const long long g = ri[kWarps * j].g_first + k;
+      if (k < ri[kWarps * j].nslot && split::group_live(g, ri[kWarps * j].T, G)) {
+        const long long slot = split::partial_slot(p, mode, g, ri[kWarps * j].s, ri[kWarps * j].i);
+        const float m = p.part_m[slot * kHeads + h];
+        M[j] = fmaxf(M[j], m);
+        if (k0 == 0) {
+          mk[j] = m;
+          lk[j] = p.part_l[slot * kHeads + h];
+          sl[j] = slot;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kRowsPerWarp; ++j) M[j] = warp_max(M[j]);
+  // (3) weighted sums, two rows at a time, partials in chunks of 32 (weights lane-held)
+#pragma unroll
+  for (int jp = 0; jp < kRowsPerWarp; jp += 2) {
+    float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+    float dsum[2] = {0.f, 0.f};
+    const int pair_max = max(ri[kWarps * jp].nslot, ri[kWarps * (jp + 1)].nslot);
+    for (int k0 = 0; k0 < pair_max; k0 += 32) {
+      float w[2];
+      long long slot[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int j = jp + e;
+        float m = mk[j], l = lk[j];
+        slot[e] = sl[j];
+        if (k0 > 0) {  // beyond the first 32 partials: load this chunk's terms
+          const int k = k0 + lane;
+          const long long g = ri[kWarps * j].g_first + k;
+          m = -INFINITY;
+          l = 0.f;
+          if (k < ri[kWarps * j].nslot && split::group_live(g, ri[kWarps * j].T, G)) {
+            slot[e] = split::partial_slot(p, mode, g, ri[kWarps * j].s, ri[kWarps * j].i);
+            m = p.part_m[slot[e] * kHeads + h];
+            l = p.part_l[slot[e] * kHeads + h];
+          }
+        }
+        w[e] = (M[j] == -INFINITY || m == -INFINITY) ? 0.f : exp2f(m - M[j]);
+        dsum[e] += w[e] * l;
+      }
+      const int cnt = min(32, pair_max - k0);
+      for (int q0 = 0; q0 < cnt; q0 += kMaxBatch) {
+        float4 x[2][kMaxBatch];
+        float wq[2][kMaxBatch];
+#pragma unroll
+        for (int q = 0; q < kMaxBatch; ++q)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int src = (q0 + q) & 31;
+            wq[e][q] = (q0 + q < cnt) ? __shfl_sync(0xffffffffu, w[e], src) : 0.f;
+            const long long so = __shfl_sync(0xffffffffu, slot[e], src);
+            x[e][q] = (wq[e][q] != 0.f)
+                          ? *reinterpret_cast<const float4 *>(p.part_o + (so * kHeads + h) * kLatent + kc * kChunk +
+                                                              4 * lane)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+        for (int q = 0; q < kMaxBatch; ++q)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            acc[e].x += wq[e][q] * x[e][q].x;
+            acc[e].y += wq[e][q] * x[e][q].y;
+            acc[e].z += wq[e][q] * x[e][q].z;
+            acc[e].w += wq[e][q] * x[e][q].w;
+          }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int j = jp + e;
+      const int t = warp + kWarps * j;
+      const int v = v0 + t;
+      const float den = warp_sum(dsum[e]);
+      const bool good = v < n && M[j] != -INFINITY && den > 0.f;
+      const float inv = good ? 1.f / den : 0.f;
+      const float4 o = make_float4(acc[e].x * inv, acc[e].y * inv, acc[e].z * inv, acc[e].w * inv);
+      const uint32_t lo = pack_bf16x2(o.x, o.y), hi = pack_bf16x2(o.z, o.w);
+      if (v < n) {
+        if (p.o_latent != nullptr)
+          *reinterpret_cast<uint2 *>(p.o_latent + ((long long)v * kHeads + h) * kLatent + kc * kChunk + 4 * lane) =
+              make_uint2(lo, hi);
+        if (p.lse != nullptr && kc == 0 && lane == 0)
+          p.lse[(long long)v * kHeads + h] = good ? (M[j] + log2f(den)) * 0.69314718055994530942f : -INFINITY;
+      }
+      // B operand: row t, latent 4*lane .. 4*lane+3 of the chunk, 128-byte swizzle
+      const int atom = lane >> 4, unit = (lane & 15) >> 1;
+      st_shared_v2(b_base + atom * kBAtomBytes + t * 128 + ((unit ^ (t & 7)) << 4) + (lane & 1) * 8, lo, hi);
+    }
   }
   fence_proxy_async_smem();  // make the B tile visible to the tensor core
   tc_fence_before();

@@ -42,7 +42,7 @@ constexpr int kOffP = kOffKV + kStages * kStageBytes;
 constexpr int kOffBar = kOffP + kPBytes;
 constexpr int kBarFull = 0, kBarEmpty = kStages, kBarSFull = 2 * kStages, kBarSEmpty = kBarSFull + 2,
               kBarPFull = kBarSEmpty + 2, kBarPEmpty = kBarPFull + 1, kBarQ = kBarPEmpty + 1, kBarO = kBarQ + 1,
-              kNumBars = kBarO + 1;
+              kBarDrain = kBarO + 1, kNumBars = kBarDrain + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar[kBarPEmpty], 1);
     mbar_init(&bar[kBarQ], 4);
     mbar_init(&bar[kBarO], 1);
+    mbar_init(&bar[kBarDrain], 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -114,6 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
+      uint32_t issued = 0;
       for (int kt = 0; kt < n_kt; ++kt) {
         const int s = kt % kStages;
         if (!mbar_wait(&bar[kBarEmpty + s], ((kt / kStages) & 1) ^ 1, abort_flag, p.status)) break;
@@ -125,7 +127,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(dst + c * kBoxBytes, &tm_k, &bar[kBarFull + s], c * 64, h, tok);
           tma_load_3d(dst + kKBytes + c * kBoxBytes, &tm_v, &bar[kBarFull + s], c * 64, h, tok);
         }
+        issued = kt + 1;
       }
+      // every issued copy lands before the CTA may exit (also after an abort)
+      if (!drain_ring(&bar[kBarFull], kStages, issued)) report_status(p.status, kStatusTimeout);
     }
   } else if (warp == 1) {
     // S[q, keys] = Q (TMEM) * K_tile^T; K_tile K-major: K step of 16 dims = 32 bytes in a
@@ -298,9 +303,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   __syncwarp();
+  // after an abort, both MMA issuers' MMAs finish before TMEM is released
+  if (warp == 6 && *abort_flag) {
+    if (lane == 0) umma_commit(&bar[kBarDrain]);
+    __syncwarp();
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    if (*abort_flag) {
+      if (lane == 0) {
+        umma_commit(&bar[kBarDrain]);
+        if (!mbar_wait_drain(&bar[kBarDrain], 0)) report_status(p.status, kStatusTimeout);
+      }
+      __syncwarp();
+    }
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

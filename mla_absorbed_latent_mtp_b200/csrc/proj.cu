@@ -99,13 +99,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       grid_dep_wait();
       const int xh = p.x_bcast ? 0 : h;
       for (int kc = 0; kc < pre; ++kc) tma_load_3d(b_stage0 + kc * b_bytes, &tm_x, &full[kc], kc * kBK, xh, nt * NT);
+      int issued = pre;
       for (int kc = pre; kc < nk; ++kc) {
         const int s = kc % kStages, use = kc / kStages;
         if (!mbar_wait(&empty[s], (use & 1) ^ 1, abort_flag, nullptr)) break;
         mbar_arrive_expect_tx(&full[s], kABytes + NT * kBK * 2);
         load_a(kc, s);
         tma_load_3d(b_stage0 + s * b_bytes, &tm_x, &full[s], kc * kBK, xh, nt * NT);
+        issued = kc + 1;
       }
+      // every issued copy lands before the CTA may exit (also after an abort)
+      drain_ring(full, (uint32_t)kStages, (uint32_t)issued);
     }
   } else if (warp == 1) {
     const uint32_t idesc = idesc_bf16_f32(kBM, NT, kAMajorMN, false);

@@ -85,6 +85,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
   }
 }
 
+// Bounded wait that ignores the CTA's abort flag, for draining copies and MMAs before a CTA
+// exits (normally or after an abort): returns false if the phase did not complete within
+// limit_cycles.
+constexpr long long kDrainLimitCycles = 20000000LL;  // about 10 ms
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity,
+                                                long long limit_cycles = kDrainLimitCycles) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_test_wait(a, parity)) return true;
+  const long long t0 = clock64();
+  while (clock64() - t0 < limit_cycles) {
+    if (mbar_try_wait_sleep(a, parity, 100000u)) return true;
+  }
+  return false;
+}
+
+// After a producer stops issuing loads into a ring of `slots` full-barriers (`issued`
+// loads in ring order, one phase per use), wait until every issued load has landed, so
+// that no copy writes shared memory after the CTA has exited.  Loads already consumed
+// pass at once.  Returns false if one did not land in time.
+__device__ __forceinline__ bool drain_ring(uint64_t *full, uint32_t slots, uint32_t issued) {
+  bool ok = true;
+  for (uint32_t rp = 0; rp < slots && rp < issued; ++rp) {
+    const uint32_t k_last = rp + slots * ((issued - 1 - rp) / slots);
+    ok = mbar_wait_drain(&full[rp], (k_last / slots) & 1) && ok;
+  }
+  return ok;
+}
+
 // One lane of the (fully active) warp is elected; the others skip.  Issuing tcgen05 MMAs
 // from the elected lane, with operands computed by the whole warp under warp-uniform control
 // flow, keeps the operands in uniform registers: no per-MMA conversion from a divergent lane.
@@ -148,6 +176,7 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint3
 }
 // Arrive on `bar` once all prior cp.async copies of this thread have landed
 // (the arrival is one of the barrier's expected arrivals).
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }

@@ -87,3 +87,12 @@ def test_prefill_flop_counts(L):
     assert f["absorbed_attention"] == 2 * f["expanded_attention"]
     assert f["expanded"] - f["expanded_attention"] == 2 * 2 * L * 512 * 64 * 256
     assert f["absorbed"] - f["absorbed_attention"] == 2 * 2 * L * 64 * 256 * 512
+
+
+@pytest.mark.parametrize("K,n_rot", [(20, 4), (20, 1), (1000, 1), (1000, 4), (3, 4), (7, 1), (1, 1)])
+def test_graph_batches_time_exactly_k_steps(K, n_rot):
+    """The timed loops replay graphs of G steps K / G times: G must divide K."""
+    G = bench.steps_per_graph(K, n_rot)
+    assert 1 <= G <= 32 and K % G == 0
+    if any(K % g == 0 and g % n_rot == 0 for g in range(1, min(K, 32) + 1)):
+        assert G % n_rot == 0

@@ -213,12 +213,20 @@ def test_length_beyond_cache_sets_index_status():
 
 
 def test_small_workspace_rejected():
+    """The binding refuses a short workspace before the call; the C ABI itself, handed one
+    directly, returns MLA_ERR_WORKSPACE and launches nothing."""
+    import ctypes
     qt = torch.zeros(1, 1, 64, 512, dtype=torch.bfloat16, device="cuda")
     cache = torch.zeros(1, 8, 512, dtype=torch.bfloat16, device="cuda")
+    o = torch.empty(1, 1, 64, 512, dtype=torch.bfloat16, device="cuda")
     ws = torch.empty(16, dtype=torch.uint8, device="cuda")
-    with pytest.raises(m.MLAError) as e:
+    with pytest.raises(ValueError, match="workspace"):
         m.mla_attend_dense(qt, cache, None, workspace=ws)
-    assert e.value.code == m.MLA_ERR_WORKSPACE
+    vp = ctypes.c_void_p
+    code = m.lib().mla_attend_dense(vp(qt.data_ptr()), vp(cache.data_ptr()), None, 1, 1, 64, 512, 8, 1.0 / 16,
+                                    vp(ws.data_ptr()), 16, vp(o.data_ptr()), None, None,
+                                    vp(torch.cuda.current_stream().cuda_stream))
+    assert code == m.MLA_ERR_WORKSPACE
 
 
 # ----------------------------------------------------------------------------- addressing, bit for bit

@@ -31,6 +31,13 @@ def device():
     torch.cuda.synchronize()
 
 
+# Scores are computed from bf16-rounded keys (expanded form) or absorbed queries (absorbed
+# form): a score moves by at most 2^-9 * scale * sum_d |q_d k_d|, about 2^-9 * 163 / 16 = 0.02
+# for unit-variance q and k over 256 dims, and the log-sum-exp by no more than its largest
+# score (a query that sees one key shows exactly that error).
+LSE_TOL = 2e-2
+
+
 def _proj_tol(ref):
     return 2.0 ** -8 * np.abs(ref) + 1e-5
 
@@ -83,9 +90,10 @@ def test_prefill_both_forms_match_oracle(B, L):
             mx, mean = errors(got[b, t], r["out"])
             assert mx <= MAX_ABS_TOL and mean <= MEAN_ABS_TOL, (name, b, t, mx, mean)
             gl = lse[b, t].cpu().numpy().astype(np.float64)
-            assert np.abs(gl - r["lse"]).max() <= 5e-3, (name, b, t)
+            assert np.abs(gl - r["lse"]).max() <= LSE_TOL, (name, b, t)
+    # the two forms round different intermediates (k, v against q~, o): they agree to the gate
     mx, mean = errors(out_e, out_a)
-    assert mx <= MAX_ABS_TOL and mean <= 1e-3, (mx, mean)
+    assert mx <= MAX_ABS_TOL and mean <= MEAN_ABS_TOL, (mx, mean)
 
 
 def test_prefill_expanded_rows_past_a_sequence_do_not_leak():
