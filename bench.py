@@ -210,7 +210,13 @@ class ClockSampler:
                 bits = int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))
             except Exception:
                 return
-            self.rows.append((time.time(), mhz, max_mhz, [n for b, n in self.NVML_REASONS if bits & b]))
+            row = (time.time(), mhz, max_mhz, [n for b, n in self.NVML_REASONS if bits & b])
+            try:  # memory clock and board power, where NVML offers them
+                row = row + (float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_MEM)),
+                             pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0)
+            except Exception:
+                pass
+            self.rows.append(row)
             time.sleep(0.001)
 
     def _read_smi(self):
@@ -242,9 +248,16 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0,
                     "source": self.source}
         reasons = sorted({n for r in window for n in r[3]})
-        return {"sm_mhz": statistics.median(r[1] for r in window), "sm_max_mhz": max(r[2] for r in window),
-                "sm_mhz_min": min(r[1] for r in window), "reasons": reasons, "samples": len(window),
-                "source": self.source}
+        out = {"sm_mhz": statistics.median(r[1] for r in window), "sm_max_mhz": max(r[2] for r in window),
+               "sm_mhz_min": min(r[1] for r in window), "reasons": reasons, "samples": len(window),
+               "source": self.source}
+        nv = [r for r in window if len(r) > 5]
+        if nv:
+            out["mem_mhz"] = statistics.median(r[4] for r in nv)
+            out["mem_mhz_min"] = min(r[4] for r in nv)
+            out["power_w_median"] = statistics.median(r[5] for r in nv)
+            out["power_w_max"] = max(r[5] for r in nv)
+        return out
 
 
 # ----------------------------------------------------------------------------- distributed helpers

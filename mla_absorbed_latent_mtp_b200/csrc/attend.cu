@@ -791,16 +791,14 @@ __global__ void __launch_bounds__(128, 4) combine_kernel(const AttendParams p, i
   const int b = v / p.Q, i = v % p.Q;
   const int s = (mode == kModeIndexed) ? v : b;
   const int tid = threadIdx.x;
-  const long long G = p.groups;
-  // The sequence's group range is block-uniform and costs 64-bit divisions: one thread
-  // computes it.  A group is empty only when there are fewer tiles than groups.
-  __shared__ long long sh_T, sh_g_first;
-  __shared__ int sh_nslot;
+  // The sequence's partials are block-uniform and cost 64-bit divisions: one thread finds
+  // them (their workspace slots, up to kMaxPartials; beyond that the range is consecutive).
+  constexpr int kMaxPartials = 256;
+  __shared__ long long sh_slot[kMaxPartials];
+  __shared__ split::GroupRange sh_gr;
   if (tid == 0) {
     const split::GroupRange gr = split::seq_group_range(p, mode, s);
-    sh_T = gr.T;
-    sh_g_first = gr.g_first;
-    sh_nslot = gr.nslot;
+    sh_gr = gr;
     if (blockIdx.y == 0 && i == 0 && mode != kModeIndexed && p.seq_lens != nullptr) {
       const int L = p.seq_lens[b];
       const int cap = (mode == kModePaged) ? p.max_pages * kPageTokens : p.Lmax;
@@ -808,9 +806,11 @@ __global__ void __launch_bounds__(128, 4) combine_kernel(const AttendParams p, i
     }
   }
   __syncthreads();
-  const long long T = sh_T, g_first = sh_g_first;
-  const int nslot = sh_nslot;
-  const bool all_live = T >= G;
+  const split::GroupRange gr = sh_gr;
+  const int nslot = gr.count;
+  for (int k = tid; k < nslot && k < kMaxPartials; k += blockDim.x)
+    sh_slot[k] = split::partial_slot(p, mode, gr.partial_group(k), s, i);
+  __syncthreads();
   const int h0 = blockIdx.y * kCombineHeads;
   const int lat = tid * 4;
   float M[kCombineHeads], den[kCombineHeads];
@@ -826,9 +826,10 @@ __global__ void __launch_bounds__(128, 4) combine_kernel(const AttendParams p, i
     float4 ok[kCombineHeads][kCombineChunk];
 #pragma unroll
     for (int j = 0; j < kCombineChunk; ++j) {
-      const long long gg = g_first + k0 + j;
-      const bool live = (k0 + j < nslot) && (all_live || split::group_live(gg, T, G));
-      const long long slot = split::partial_slot(p, mode, gg, s, i);
+      const int k = k0 + j;
+      const bool live = k < nslot;
+      const long long slot =
+          !live ? 0 : (k < kMaxPartials ? sh_slot[k] : split::partial_slot(p, mode, gr.partial_group(k), s, i));
 #pragma unroll
       for (int hh = 0; hh < kCombineHeads; ++hh) {
         const long long row = slot * kRows + h0 + hh;

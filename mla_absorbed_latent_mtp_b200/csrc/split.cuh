@@ -22,36 +22,43 @@ __device__ __forceinline__ int num_seqs(const AttendParams &p, int mode) {
 
 __device__ __forceinline__ long long group_start(long long g, long long T, long long G) { return g * T / G; }
 
-// The range of groups that processed tiles of sequence s, from the table the attend kernel
-// wrote: groups g_first .. g_first + nslot - 1 (nslot = 0 for a sequence without tiles).
-// T is the total tile count.  A group inside the range holds no tiles of s only when there
-// are fewer tiles than groups (then some groups are empty).
+// The group whose tile range holds tile t: the largest g with g*T/G <= t.
+__device__ __forceinline__ long long group_of(long long t, long long T, long long G) { return ((t + 1) * G - 1) / T; }
+
+// The partials of sequence s, from the table the attend kernel wrote: `count` groups, the
+// k-th being partial_group(k).  With at least as many tiles as groups (T >= G) every group
+// holds tiles and the sequence's partials are those of the consecutive groups
+// g_first .. g_first + count - 1; with fewer tiles than groups every group holds at most one
+// tile, so the k-th partial is the group of the sequence's k-th tile (enumerating the
+// groups in between would visit mostly empty ones).
 struct GroupRange {
-  long long g_first;
-  long long T;
-  int nslot;
+  long long g_first;  // first group (T >= G)
+  long long ts;       // first tile of the sequence
+  long long T, G;
+  int count;          // number of partials
+  __device__ __forceinline__ long long partial_group(int k) const {
+    return T >= G ? g_first + k : group_of(ts + k, T, G);
+  }
 };
 
 __device__ __forceinline__ GroupRange seq_group_range(const AttendParams &p, int mode, int s) {
   const int ns = num_seqs(p, mode);
-  const long long G = p.groups;
   GroupRange r;
+  r.G = p.groups;
   r.T = p.seq_ts[ns - 1] + p.seq_nt[ns - 1];
-  const long long ts = p.seq_ts[s];
+  r.ts = p.seq_ts[s];
   const int nt = p.seq_nt[s];
-  long long g_last = -1;
   r.g_first = 0;
+  r.count = 0;
   if (nt > 0) {
-    r.g_first = ((ts + 1) * G - 1) / r.T;
-    g_last = ((ts + nt) * G - 1) / r.T;
+    if (r.T >= r.G) {
+      r.g_first = group_of(r.ts, r.T, r.G);
+      r.count = (int)(group_of(r.ts + nt - 1, r.T, r.G) - r.g_first + 1);
+    } else {
+      r.count = nt;
+    }
   }
-  r.nslot = (int)(g_last - r.g_first + 1);
   return r;
-}
-
-// Whether group g holds any tiles (always true when every group has tiles).
-__device__ __forceinline__ bool group_live(long long g, long long T, long long G) {
-  return T >= G || group_start(g, T, G) < group_start(g + 1, T, G);
 }
 
 // Workspace slot of the partial of group g, tile-list sequence s, query i.
