@@ -43,7 +43,7 @@ constexpr int kSlotBytes = 2 * kAtomBytes;      // 16 KB: 64 rows x 128 latent
 constexpr int kQtChunks = kLatent / 64;
 constexpr int kQtChunkBytes = kRows * 64 * 2;   // 8 KB: 64 heads x 64 latent
 constexpr int kPBytes = kTile * kRows * 2;      // 8 KB: P^T, 64 rows x 64 heads (bf16)
-constexpr int kThreads = 352;  // producer, score MMA, 8 softmax warps, value MMA
+constexpr int kThreads = 384;  // producer, score MMA, 8 softmax warps, value MMA, second gather warp
 constexpr int kSoftmaxWarps = 8;
 constexpr float kTau = 8.0f;  // lazy rescale: the running max is raised only when a score
                               // exceeds it by more than 2^8 (probabilities stay <= 256)
@@ -223,8 +223,10 @@ __device__ __forceinline__ uint32_t ring_use(uint32_t k) { return k / kSlots; }
 // ------------------------------------------------------------------ producer (warp 0)
 // Issues the loads; counts the q~ loads and the ring-slot loads it issued (for the drain).
 template <int kMode>
+// Index lists are gathered by two warps (half 0: warp 0, tile rows 0-31 and the q~ loads;
+// half 1: warp 11, tile rows 32-63); dense and paged tiles by lane 0 of warp 0 (half 0).
 __device__ void producer_loads(const AttendParams &p, const Shared &sh, const CUtensorMap *tm_cache,
-                               const CUtensorMap *tm_qt, int iq, long long t0, long long t1, int lane,
+                               const CUtensorMap *tm_qt, int iq, long long t0, long long t1, int lane, int half,
                                uint32_t &q_use, uint32_t &slots_issued) {
   uint64_t *bar = sh.bar;
   uint32_t tile_k = 0;
@@ -235,56 +237,53 @@ __device__ void producer_loads(const AttendParams &p, const Shared &sh, const CU
     const int b = (kMode == kModeIndexed) ? sg.s / p.Q : sg.s;
     const int qi = (kMode == kModeIndexed) ? sg.s % p.Q : iq;
     const int qrow0 = (b * p.Q + qi) * kRows;
-    bool ok;
-    if constexpr (kMode == kModeIndexed)
-      ok = wait_warp(&bar[kBarQEmpty], (q_use & 1) ^ 1, sh, p.status);  // whole warp runs this role
-    else
-      ok = mbar_wait(&bar[kBarQEmpty], (q_use & 1) ^ 1, sh.abort_flag, p.status);  // lane 0 only
-    if (!ok) return;
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&bar[kBarQFull], kQtChunks * kQtChunkBytes);
+    if (half == 0) {
+      bool ok;
+      if constexpr (kMode == kModeIndexed)
+        ok = wait_warp(&bar[kBarQEmpty], (q_use & 1) ^ 1, sh, p.status);  // whole warp runs this role
+      else
+        ok = mbar_wait(&bar[kBarQEmpty], (q_use & 1) ^ 1, sh.abort_flag, p.status);  // lane 0 only
+      if (!ok) return;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bar[kBarQFull], kQtChunks * kQtChunkBytes);
 #pragma unroll
-      for (int c = 0; c < kQtChunks; ++c) tma_load_2d(sh.qt(c), tm_qt, &bar[kBarQFull], c * 64, qrow0);
-    }
-    ++q_use;
-    // indexed: the list entries of the next tile are read while this tile's rows are
-    // copied (two rows per lane), so the index load latency is off the copy path
-    const int32_t *list = p.indices + ((long long)b * p.Q + qi) * p.K;
-    int nxt[2] = {0, 0};
-    if constexpr (kMode == kModeIndexed) {
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const int k = sg.lo * kTile + lane + 32 * m;
-        if (k < p.K) nxt[m] = list[k];
+        for (int c = 0; c < kQtChunks; ++c) tma_load_2d(sh.qt(c), tm_qt, &bar[kBarQFull], c * 64, qrow0);
       }
+      ++q_use;
+    }
+    // indexed: the list entry of this lane's row of the next tile is read while this
+    // tile's rows are copied, so the index load latency is off the copy path
+    const int32_t *list = p.indices + ((long long)b * p.Q + qi) * p.K;
+    const int row_lane = 32 * half + lane;  // the tile row whose list entry this lane holds
+    int nxt = 0;
+    if constexpr (kMode == kModeIndexed) {
+      const int k = sg.lo * kTile + row_lane;
+      if (k < p.K) nxt = list[k];
     }
     for (int t = sg.lo; t < sg.hi; ++t, ++tile_k) {
       if constexpr (kMode == kModeIndexed) {
-        // two tile rows per lane; rows past the list end are zero-filled
+        // rows past the list end are zero-filled
         const int limit = query_limit(p, b, qi);
-        const int cur[2] = {nxt[0], nxt[1]};
+        const int cur = nxt;
         if (t + 1 < sg.hi) {
-#pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            const int k = (t + 1) * kTile + lane + 32 * m;
-            if (k < p.K) nxt[m] = list[k];
-          }
+          const int k = (t + 1) * kTile + row_lane;
+          if (k < p.K) nxt = list[k];
         }
-        // cache row (in units of R) of the tile rows lane and lane + 32, -1 when unused
-        int rowi[2];
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          const int k = t * kTile + lane + 32 * m;
+        // cache row (in units of R) of tile row row_lane, -1 when unused
+        int rowi;
+        {
+          const int k = t * kTile + row_lane;
           bool bad = false;
           long long row = 0;
-          const bool used = k < p.K && cur[m] != kUnusedEntry;
-          if (used) row = indexed_row_of(b, cur[m], p.Lmax, limit, bad);
+          const bool used = k < p.K && cur != kUnusedEntry;
+          if (used) row = indexed_row_of(b, cur, p.Lmax, limit, bad);
           if (bad) report_status(p.status, kStatusIndex);
-          rowi[m] = (used && !bad) ? (int)row : -1;
+          rowi = (used && !bad) ? (int)row : -1;
         }
         // Each copy instruction moves two tile rows' 256-byte slice of this slot: lanes
         // 0-15 row 2i, lanes 16-31 row 2i + 1, 16 bytes each, so every instruction reads four
-        // whole 128-byte lines (B * Lmax < 2^31 rows, so a row fits an int).
+        // whole 128-byte lines (B * Lmax < 2^31 rows, so a row fits an int).  This warp's
+        // half of the slot is its 32 rows.
         const int u = lane & 15, at = u >> 3, pc = u & 7;
         for (int qq = 0; qq < kSlotQuarters; ++qq) {
           const uint32_t k = tile_k * kSlotQuarters + qq;
@@ -293,9 +292,9 @@ __device__ void producer_loads(const AttendParams &p, const Shared &sh, const CU
           const uint32_t dst_s = smem_u32(sh.slot(rp)) + at * kAtomBytes;
           const uint16_t *src_q = p.cache + qq * 128 + at * 64 + pc * 8;
 #pragma unroll
-          for (int i = 0; i < kTile / 2; ++i) {
-            const int r = 2 * i + (lane >> 4);
-            const int ri = __shfl_sync(0xffffffffu, rowi[i >> 4], r & 31);
+          for (int i = 0; i < kTile / 4; ++i) {
+            const int r = 32 * half + 2 * i + (lane >> 4);
+            const int ri = __shfl_sync(0xffffffffu, rowi, r & 31);
             cp_async_16(dst_s + r * 128 + ((pc ^ (r & 7)) << 4), src_q + (long long)max(ri, 0) * kLatent,
                         ri >= 0 ? 16u : 0u);
           }
@@ -330,9 +329,9 @@ __device__ void producer_loads(const AttendParams &p, const Shared &sh, const CU
 // issued has landed.
 template <int kMode>
 __device__ void producer_role(const AttendParams &p, const Shared &sh, const CUtensorMap *tm_cache,
-                              const CUtensorMap *tm_qt, int iq, long long t0, long long t1, int lane) {
+                              const CUtensorMap *tm_qt, int iq, long long t0, long long t1, int lane, int half) {
   uint32_t q_use = 0, slots_issued = 0;
-  producer_loads<kMode>(p, sh, tm_cache, tm_qt, iq, t0, t1, lane, q_use, slots_issued);
+  producer_loads<kMode>(p, sh, tm_cache, tm_qt, iq, t0, t1, lane, half, q_use, slots_issued);
   if constexpr (kMode == kModeIndexed) cp_async_wait_all();  // this lane's row copies
   if (lane == 0) {
     bool ok = drain_ring(&sh.bar[kBarQFull], 1, q_use);
@@ -703,7 +702,7 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     for (int c = 0; c < kSlots; ++c) {
-      mbar_init(&sh.bar[kBarCFull + c], kMode == kModeIndexed ? 32 : 1);
+      mbar_init(&sh.bar[kBarCFull + c], kMode == kModeIndexed ? 64 : 1);  // indexed: 2 warps of copies
       mbar_init(&sh.bar[kBarCEmpty + c], 1);
     }
     mbar_init(&sh.bar[kBarQFull], 1);
@@ -741,7 +740,9 @@ __global__ void __launch_bounds__(384, 1)
       prefetch_tensormap(&tm_qt);
       if (kMode != kModeIndexed) prefetch_tensormap(&tm_cache);
     }
-    if (kMode == kModeIndexed || lane == 0) producer_role<kMode>(p, sh, &tm_cache, &tm_qt, iq, t0, t1, lane);
+    if (kMode == kModeIndexed || lane == 0) producer_role<kMode>(p, sh, &tm_cache, &tm_qt, iq, t0, t1, lane, 0);
+  } else if (warp == 11) {
+    if (kMode == kModeIndexed) producer_role<kMode>(p, sh, &tm_cache, &tm_qt, iq, t0, t1, lane, 1);
   } else if (warp == 1) {
     score_mma_role<kMode>(p, sh, tmem, iq, t0, t1, lane);
   } else if (warp == 10) {
