@@ -45,6 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TRAFFIC = {
     ("dense_decode", "2f78743fc2d4f68e"): 277_555_968,
     ("mtp_verify", "2f78743fc2d4f68e"): 556_532_480,
+    ("indexed_sparse_decode", "4510330f24d2dff0"): 71_969_280,
 }
 
 
