@@ -43,9 +43,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one attend launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
 # ncu capture summarised in profiles/, keyed by the hash of the kernel source it was taken on.
 TRAFFIC = {
-    ("dense_decode", "2f78743fc2d4f68e"): 277_555_968,
-    ("mtp_verify", "2f78743fc2d4f68e"): 556_532_480,
-    ("indexed_sparse_decode", "4510330f24d2dff0"): 71_969_280,
+    ("tiny_dense_decode", "ee633b89767f85fc"): 398_080,
+    ("dense_decode", "ee633b89767f85fc"): 277_656_832,
+    ("mtp_verify", "ee633b89767f85fc"): 556_562_432,
+    ("ragged_paged_decode", "ee633b89767f85fc"): 4_379_875_072,
+    ("indexed_sparse_decode", "ee633b89767f85fc"): 71_918_592,
 }
 
 
@@ -149,7 +151,7 @@ def load_peaks():
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for fn in ("attend.cu", "sm100.cuh", "internal.h"):
+    for fn in ("attend.cu", "sm100.cuh", "split.cuh", "internal.h"):
         with open(os.path.join(ROOT, "mla_absorbed_latent_mtp_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

@@ -71,10 +71,14 @@ def test_workload_bounds_are_the_expected_ones():
 
 
 def test_recorded_traffic_is_close_to_the_algorithmic_bytes():
-    """A recorded DRAM traffic figure well above the cache bytes would mean re-reads."""
+    """A recorded DRAM traffic figure well above the cache bytes would mean re-reads.  Allowed
+    on top of 10%: q~ (64 KiB per query row, read once) and 128 KiB of fixed per-launch reads
+    (lengths, tables, tensor maps), which dominate only the tiny workload."""
     for (name, _src), traffic in bench.TRAFFIC.items():
-        cache = bench.step_bytes(synth.make_workload(name, with_data=False))["cache"]
-        assert cache <= traffic <= 1.1 * cache, (name, traffic, cache)
+        wl = synth.make_workload(name, with_data=False)
+        cache = bench.step_bytes(wl)["cache"]
+        qt = wl.B * wl.Q * 64 * 512 * 2
+        assert cache <= traffic <= 1.1 * cache + qt + (1 << 17), (name, traffic, cache)
 
 
 @pytest.mark.parametrize("L", [1, 5, 64, 130])
