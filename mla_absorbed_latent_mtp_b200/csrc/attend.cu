@@ -777,15 +777,16 @@ __global__ void __launch_bounds__(384, 1)
 // ------------------------------------------------------------------ combine
 // One block per (query row v = b * Q + i) and pair of heads; thread t owns latent 4t..4t+3
 // of both heads.  The partials of the CTA groups that processed tiles of the row's
-// sequence are merged online in chunks of six (every partial of the benchmark shapes in
-// one chunk), all loads of a chunk in flight at once:
+// sequence are merged online in chunks of three, all loads of a chunk in flight at once
+// (chunks this small keep a thread at 64 registers, so eight blocks fit on an SM and the
+// 1,024 blocks of a 32-row step run in one wave):
 // with M the largest running max so far, O = sum 2^(m_g - M) O_g and l = sum 2^(m_g - M) l_g,
 // then O / l and lse = M + log2 l.  The sequence's place in the tile list comes from the
 // table the attend kernel wrote.
 constexpr int kCombineHeads = 2;
-constexpr int kCombineChunk = 6;
+constexpr int kCombineChunk = 3;
 
-__global__ void __launch_bounds__(128, 4) combine_kernel(const AttendParams p, int mode) {
+__global__ void __launch_bounds__(128, 8) combine_kernel(const AttendParams p, int mode) {
   grid_dep_launch();
   grid_dep_wait();  // the partials come from the attend kernel just before
   const int v = blockIdx.x;  // b * Q + i
