@@ -636,16 +636,18 @@ def measure_config(name, args, device, rank, world, clocks, peaks, peak_kind, sr
     # likewise.
     Kb = max(len(idx_sets), min(K, 50) // len(idx_sets) * len(idx_sets))
 
-    def timed_graph(fn, reps):
+    def timed_graph(fn, reps, replays=3):
+        # the average call over `replays` back-to-back replays of a graph of `reps` calls
         g = capture(fn, reps, idx_turn)
         g.replay()
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        g.replay()
+        for _ in range(replays):
+            g.replay()
         b.record()
         torch.cuda.synchronize()
-        return a.elapsed_time(b) / reps
+        return a.elapsed_time(b) / (reps * replays)
 
     stage = reduce_max([timed_graph(absorb, Kb), timed_graph(attend, Kb), timed_graph(up, Kb)], device)
     aw0 = time.time()
