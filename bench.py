@@ -43,11 +43,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one attend launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
 # ncu capture summarised in profiles/, keyed by the hash of the kernel source it was taken on.
 TRAFFIC = {
-    ("tiny_dense_decode", "ee633b89767f85fc"): 398_080,
-    ("dense_decode", "ee633b89767f85fc"): 277_656_832,
-    ("mtp_verify", "ee633b89767f85fc"): 556_562_432,
-    ("ragged_paged_decode", "ee633b89767f85fc"): 4_379_875_072,
-    ("indexed_sparse_decode", "ee633b89767f85fc"): 71_918_592,
+    ("tiny_dense_decode", "e365173f9ea1c4d7"): 398_336,
+    ("dense_decode", "e365173f9ea1c4d7"): 278_236_160,
+    ("mtp_verify", "e365173f9ea1c4d7"): 558_177_280,
+    ("ragged_paged_decode", "e365173f9ea1c4d7"): 4_379_070_720,
+    ("indexed_sparse_decode", "e365173f9ea1c4d7"): 72_137_216,
 }
 
 
