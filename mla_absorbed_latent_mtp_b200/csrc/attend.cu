@@ -597,6 +597,22 @@ __device__ void softmax_role(const AttendParams &p, const Shared &sh, uint32_t t
             m_reg[2 * j + e] = m_used[c];
           }
       }
+      // probabilities, rounded to bf16 for the value product; l sums the rounded values.
+      // They are computed into registers first: the wait for this P buffer (the value
+      // product of tile n-2) then overlaps the exponentials instead of preceding them.
+      uint32_t pw[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // h = 0: row r0, h = 1: row r0 + 8
+          const float x0 = s2[4 * j + 2 * h], x1 = s2[4 * j + 2 * h + 1];
+          const float p0 = (x0 == -INFINITY) ? 0.f : fast_exp2(x0 - m_reg[2 * j]);
+          const float p1 = (x1 == -INFINITY) ? 0.f : fast_exp2(x1 - m_reg[2 * j + 1]);
+          const uint32_t w = pack_bf16x2(p0, p1);
+          l_part[2 * j] += bf16lo_to_f32(w);
+          l_part[2 * j + 1] += bf16hi_to_f32(w);
+          pw[2 * j + h] = w;
+        }
       // this P buffer is free (the value product of tile n-2 has finished)
       mbar_wait(&bar[kBarPEmpty + sb], ((n >> 1) & 1) ^ 1, sh.abort_flag, p.status);
       if (any && t > sg.lo) {
@@ -616,21 +632,12 @@ __device__ void softmax_role(const AttendParams &p, const Shared &sh, uint32_t t
         }
         tmem_st_wait();
       }
-      // probabilities, rounded to bf16 for the value product; l sums the rounded values
       const uint32_t pb = smem_u32(sh.pbuf(sb)) + p_off;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint32_t sw = (uint32_t)(((wg * 4 + j) ^ (r0 & 7)) << 4);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {  // h = 0: row r0, h = 1: row r0 + 8
-          const float x0 = s2[4 * j + 2 * h], x1 = s2[4 * j + 2 * h + 1];
-          const float p0 = (x0 == -INFINITY) ? 0.f : fast_exp2(x0 - m_reg[2 * j]);
-          const float p1 = (x1 == -INFINITY) ? 0.f : fast_exp2(x1 - m_reg[2 * j + 1]);
-          const uint32_t w = pack_bf16x2(p0, p1);
-          l_part[2 * j] += bf16lo_to_f32(w);
-          l_part[2 * j + 1] += bf16hi_to_f32(w);
-          st_shared_b32(pb + h * 8 * 128 + sw, w);
-        }
+        for (int h = 0; h < 2; ++h) st_shared_b32(pb + h * 8 * 128 + sw, pw[2 * j + h]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
