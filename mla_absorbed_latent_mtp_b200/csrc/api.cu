@@ -122,10 +122,10 @@ static mla_status attend_common(int mode, const uint16_t *q_tilde, const uint16_
   CUtensorMap tm_cache, tm_qt;
   {
     const uint64_t rows = (mode == kModePaged) ? (uint64_t)num_pages * kPageTokens : (uint64_t)B * Lmax;
-    const uint64_t dims[2] = {(uint64_t)R, rows};
-    const uint64_t strides[1] = {(uint64_t)R * 2};
-    const uint32_t box[2] = {64, 64};
-    if (!make_map(&tm_cache, cache, 2, dims, strides, box)) return cuda_status(cudaErrorInvalidValue);
+    const uint64_t dims[3] = {64, rows, (uint64_t)R / 64};
+    const uint64_t strides[2] = {(uint64_t)R * 2, 128};
+    const uint32_t box[3] = {64, 64, 2};
+    if (!make_map(&tm_cache, cache, 3, dims, strides, box)) return cuda_status(cudaErrorInvalidValue);
   }
   {
     const uint64_t dims[2] = {(uint64_t)R, (uint64_t)B * Q * H};

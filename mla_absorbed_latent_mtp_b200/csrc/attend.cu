@@ -316,8 +316,8 @@ __device__ void producer_loads(const AttendParams &p, const Shared &sh, const CU
           const uint32_t rp = ring_pos(k);
           if (!mbar_wait(&bar[kBarCEmpty + rp], (ring_use(k) & 1) ^ 1, sh.abort_flag, p.status)) return;
           mbar_arrive_expect_tx(&bar[kBarCFull + rp], kSlotBytes);
-          tma_load_2d(sh.slot(rp), tm_cache, &bar[kBarCFull + rp], qq * 128, (int)row);
-          tma_load_2d(sh.slot(rp) + kAtomBytes, tm_cache, &bar[kBarCFull + rp], qq * 128 + 64, (int)row);
+          // one copy per slot: a 3-D box {64 latent, 64 rows, 2 chunks} lands as the slot's two atoms
+          tma_load_3d(sh.slot(rp), tm_cache, &bar[kBarCFull + rp], 0, (int)row, 2 * qq);
           slots_issued = k + 1;
         }
       }
