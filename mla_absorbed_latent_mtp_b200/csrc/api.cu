@@ -121,6 +121,9 @@ static mla_status attend_common(int mode, const uint16_t *q_tilde, const uint16_
 
   CUtensorMap tm_cache, tm_qt;
   {
+    // cache rows seen as {64 latent, rows, R/64 chunks of 64 latent} (strides 1,024 and 128
+    // bytes): one box {64, 64, 2} is a ring slot, 64 rows x 128 latent, landing as two
+    // 128-byte-swizzled 64 x 64 atoms -- one copy per slot instead of two
     const uint64_t rows = (mode == kModePaged) ? (uint64_t)num_pages * kPageTokens : (uint64_t)B * Lmax;
     const uint64_t dims[3] = {64, rows, (uint64_t)R / 64};
     const uint64_t strides[2] = {(uint64_t)R * 2, 128};
