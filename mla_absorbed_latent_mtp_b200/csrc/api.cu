@@ -131,10 +131,12 @@ static mla_status attend_common(int mode, const uint16_t *q_tilde, const uint16_
     if (!make_map(&tm_cache, cache, 3, dims, strides, box)) return cuda_status(cudaErrorInvalidValue);
   }
   {
-    const uint64_t dims[2] = {(uint64_t)R, (uint64_t)B * Q * H};
-    const uint64_t strides[1] = {(uint64_t)R * 2};
-    const uint32_t box[2] = {64, 64};
-    if (!make_map(&tm_qt, q_tilde, 2, dims, strides, box)) return cuda_status(cudaErrorInvalidValue);
+    // q~ rows (one per head) the same way: one box {64, 64 heads, 8 chunks} is a query's
+    // whole q~, eight 64 x 64 atoms
+    const uint64_t dims[3] = {64, (uint64_t)B * Q * H, (uint64_t)R / 64};
+    const uint64_t strides[2] = {(uint64_t)R * 2, 128};
+    const uint32_t box[3] = {64, 64, (uint32_t)R / 64};
+    if (!make_map(&tm_qt, q_tilde, 3, dims, strides, box)) return cuda_status(cudaErrorInvalidValue);
   }
   AttendParams p;
   p.seq_lens = seq_lens;

@@ -246,8 +246,7 @@ __device__ void producer_loads(const AttendParams &p, const Shared &sh, const CU
       if (!ok) return;
       if (lane == 0) {
         mbar_arrive_expect_tx(&bar[kBarQFull], kQtChunks * kQtChunkBytes);
-#pragma unroll
-        for (int c = 0; c < kQtChunks; ++c) tma_load_2d(sh.qt(c), tm_qt, &bar[kBarQFull], c * 64, qrow0);
+        tma_load_3d(sh.qt(0), tm_qt, &bar[kBarQFull], 0, qrow0, 0);  // all 8 chunks in one copy
       }
       ++q_use;
     }
