@@ -43,11 +43,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one attend launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
 # ncu capture summarised in profiles/, keyed by the hash of the kernel source it was taken on.
 TRAFFIC = {
-    ("tiny_dense_decode", "e365173f9ea1c4d7"): 398_336,
-    ("dense_decode", "e365173f9ea1c4d7"): 278_236_160,
-    ("mtp_verify", "e365173f9ea1c4d7"): 558_177_280,
-    ("ragged_paged_decode", "e365173f9ea1c4d7"): 4_379_070_720,
-    ("indexed_sparse_decode", "e365173f9ea1c4d7"): 72_137_216,
+    ("tiny_dense_decode", "b314787e7e60d59f"): 398_080,
+    ("dense_decode", "b314787e7e60d59f"): 277_406_976,
+    ("mtp_verify", "b314787e7e60d59f"): 556_431_360,
+    ("ragged_paged_decode", "b314787e7e60d59f"): 4_378_591_488,
+    ("indexed_sparse_decode", "b314787e7e60d59f"): 72_119_040,
 }
 
 
