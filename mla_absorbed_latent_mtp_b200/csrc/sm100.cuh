@@ -1,5 +1,5 @@
 // sm100.cuh -- thin inline-PTX wrappers for the Blackwell (sm_100a) features the
-// kernels use: mbarriers with bounded waits, TMA tensor loads (no multicast),
+// kernels use: mbarriers with bounded waits, TMA tensor loads (each into the issuing CTA),
 // 16-byte async copies, the tcgen05 tensor-core family (TMEM allocation, MMA with
 // shared-memory descriptors issued from an elected lane, commit, TMEM loads/stores),
 // named barriers, and programmatic dependent launch (griddepcontrol).
