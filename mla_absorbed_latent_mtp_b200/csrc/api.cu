@@ -150,8 +150,14 @@ static mla_status attend_common(int mode, const uint16_t *q_tilde, const uint16_
   p.num_pages = num_pages;
   p.K = K;
   if (mode == kModeIndexed) {
+    // Every list has the same tile count, so a group count that is a multiple of the number
+    // of lists splits each list into equal parts and no CTA straddles two lists (one
+    // segment, one epilogue, one q~ load per CTA), at the price of some idle SMs.
     p.group_size = 1;
-    p.groups = sms;
+    const int lists = B * Q;
+    const int nt = (K + 63) / 64;
+    const int per_list = std::min(sms / lists, nt);
+    p.groups = per_list >= 1 ? per_list * lists : sms;
   } else {
     p.group_size = Q;
     p.groups = std::max(1, sms / Q);

@@ -66,9 +66,15 @@ def _ramp_tile(h, b, n_tiles):
     return (h * 37 + b * 11) % max(n_tiles - 4, 1)
 
 
-def _groups(mode, Q):
+def _groups(mode, B, Q, K):
+    """The kernel's CTA-group count: for index lists (all of the same length) a multiple of
+    the number of lists, so that no group straddles two lists; else SMs / Q."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    return sms if mode == "indexed" else max(1, sms // Q)
+    if mode != "indexed":
+        return max(1, sms // Q)
+    lists, nt = B * Q, (K + 63) // 64
+    per_list = min(sms // lists, nt)
+    return per_list * lists if per_list >= 1 else sms
 
 
 def _interior_steps(tile_lists, G):
@@ -178,7 +184,7 @@ def test_rescale_branch_against_oracle(mode, Q, lens, K):
     tiles = _plant(wl, Q)
     qt = _qtilde(B, Q, seed=43 + B)
     # the ramps must reach the branch: steps inside a segment, after its first tile
-    interior = _interior_steps(tiles, _groups(mode, Q))
+    interior = _interior_steps(tiles, _groups(mode, B, Q, K))
     assert interior >= 32, interior
     # and the planted scores really are the margins stated above (log2 units, fp64)
     if mode == "indexed":
