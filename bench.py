@@ -47,7 +47,7 @@ TRAFFIC = {
     ("dense_decode", "82793ecca19a9a3d"): 277_406_976,
     ("mtp_verify", "82793ecca19a9a3d"): 556_431_360,
     ("ragged_paged_decode", "82793ecca19a9a3d"): 4_378_591_488,
-    ("indexed_sparse_decode", "82793ecca19a9a3d"): 72_119_040,
+    ("indexed_sparse_decode", "82793ecca19a9a3d"): 71_430_912,
 }
 
 
