@@ -11,11 +11,11 @@
 // partial (O, running max m, running sum l) in the workspace; the combine kernel merges
 // them with their log-sum-exp weights.
 //
-// Per CTA (352 threads): warp 0 loads (TMA for dense/paged rows and q~, 16-byte async
-// copies for indexed rows), warp 1 issues the score MMAs and warp 10 the value MMAs
-// (tcgen05), warps 2-9 run the softmax and the epilogue as two warpgroups of 32 head
-// columns each.  The 64 query rows (heads) of
-// one query sit on the MMA N side and the 64 cache rows of a tile on the M side:
+// Per CTA (384 threads): warp 0 loads (one TMA copy per ring slot for dense/paged rows,
+// one for q~; 16-byte async copies for indexed rows, shared with warp 11), warp 1 issues
+// the score MMAs and warp 10 the value MMAs (tcgen05), warps 2-9 run the softmax and the
+// epilogue as two warpgroups of 32 head columns each.  The 64 query rows (heads) of one
+// query sit on the MMA N side and the 64 cache rows of a tile on the M side:
 //   S^T[tile rows, heads]  = C_tile (64 x 512, K-major)  *  Q~^T           (TMEM, fp32)
 //   O^T[latent, heads]    += C_tile^T (512 x 64, MN-major) * P^T           (TMEM, fp32)
 // so the latent dimension of O lives in TMEM lanes (4 blocks x 64 columns).  A tile
