@@ -730,6 +730,23 @@ __global__ void __launch_bounds__(384, 1)
     tmem_relinquish();
   }
   grid_dep_launch();
+  if (kMode == kModeDense && p.group_size == 1 && threadIdx.x == 0) {
+    // Decode (one query per sequence), while the previous kernel finishes: bring this
+    // CTA's first two tiles into L2, at the place they would be if every sequence held
+    // Lmax rows.  (A verify group's CTAs share their tiles; there the extra requests cost
+    // more than the early start gains.)  It reads nothing: a wrong
+    // guess (shorter sequences) costs a wasted prefetch, and every prefetched row lies in
+    // the cache ([B, Lmax] rows).  Data written by an earlier kernel is not at risk: L2 is
+    // where those writes land.
+    const long long nt = (p.Lmax + kTile - 1) / kTile;
+    const long long T_est = (long long)p.B * nt;
+    const long long t0 = group_start(g, T_est, p.groups);
+    if (t0 < T_est) {
+      const long long s = t0 / nt, j = (t0 % nt) * kTile;
+      const long long rows = min((long long)2 * kTile, (long long)p.Lmax - j);
+      bulk_prefetch_l2(p.cache + (s * p.Lmax + j) * kLatent, (uint32_t)(rows * kLatent * 2));
+    }
+  }
   grid_dep_wait();  // inputs (q~, lengths, tables, cache) may come from the previous kernel
   // tile range of this CTA's group
   const long long T = warp_total_tiles(p, kMode, lane);
