@@ -43,11 +43,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one attend launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
 # ncu capture summarised in profiles/, keyed by the hash of the kernel source it was taken on.
 TRAFFIC = {
-    ("tiny_dense_decode", "0bf1b05e0fc08753"): 398_080,
-    ("dense_decode", "0bf1b05e0fc08753"): 277_406_976,
-    ("mtp_verify", "0bf1b05e0fc08753"): 556_431_360,
-    ("ragged_paged_decode", "0bf1b05e0fc08753"): 4_378_591_488,
-    ("indexed_sparse_decode", "0bf1b05e0fc08753"): 71_430_912,
+    ("tiny_dense_decode", "9077dbfc0e8788c9"): 398_336,
+    ("dense_decode", "9077dbfc0e8788c9"): 277_510_912,
+    ("mtp_verify", "9077dbfc0e8788c9"): 556_568_576,
+    ("ragged_paged_decode", "9077dbfc0e8788c9"): 4_378_402_304,
+    ("indexed_sparse_decode", "9077dbfc0e8788c9"): 71_651_072,
 }
 
 
