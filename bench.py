@@ -43,11 +43,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one attend launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
 # ncu capture summarised in profiles/, keyed by the hash of the kernel source it was taken on.
 TRAFFIC = {
-    ("tiny_dense_decode", "9077dbfc0e8788c9"): 398_336,
-    ("dense_decode", "9077dbfc0e8788c9"): 277_510_912,
-    ("mtp_verify", "9077dbfc0e8788c9"): 556_568_576,
-    ("ragged_paged_decode", "9077dbfc0e8788c9"): 4_378_402_304,
-    ("indexed_sparse_decode", "9077dbfc0e8788c9"): 71_651_072,
+    ("tiny_dense_decode", "3a31264b08832ba4"): 398_080,
+    ("dense_decode", "3a31264b08832ba4"): 277_780_480,
+    ("mtp_verify", "3a31264b08832ba4"): 556_406_016,
+    ("ragged_paged_decode", "3a31264b08832ba4"): 4_378_480_640,
+    ("indexed_sparse_decode", "3a31264b08832ba4"): 71_251_456,
 }
 
 
@@ -122,14 +122,13 @@ def arm_config(wl, name, world) -> dict:
             "l2": l2}
 
 
-def attend_roofline(acc, att_ms, peaks, peak_kind, traffic):
-    """Roofline of attend + combine: bound by whichever of the cache bytes at the HBM peak
-    and the attend FLOPs at the bf16 tensor peak takes longer; achieved = that quantity
-    over the measured duration ``att_ms`` (milliseconds)."""
+def attend_roofline(acc, att_ms, peaks, peak_kind, traffic, kernel="attend_kernel + combine_kernel (mla_attend_*)"):
+    """Roofline of the attend call (attend + split-L merge): bound by whichever of the cache
+    bytes at the HBM peak and the attend FLOPs at the bf16 tensor peak takes longer;
+    achieved = that quantity over the measured duration ``att_ms`` (milliseconds)."""
     t_mem = acc["cache"] / (peaks["hbm_gbs"] * 1e9)
     t_tc = acc["flops_attend"] / (peaks["bf16_tflops"] * 1e12)
-    common = {"traffic": traffic, "kernel": "attend_kernel + combine_kernel (mla_attend_*)",
-              "peak_source": peak_kind}
+    common = {"traffic": traffic, "kernel": kernel, "peak_source": peak_kind}
     if t_tc > t_mem:
         ach = acc["flops_attend"] / (att_ms * 1e-3) / 1e12
         return {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -488,17 +487,40 @@ def steps_per_graph(K, n_rot=1, cap=32):
     return max(rot) if rot else max(divisors)
 
 
-def capture(fn, n, idx_turn=None):
+def capture(fn, n, idx_turn=None, keep=False):
     """A CUDA graph of n calls of fn (the library's launches go to torch's capture stream).
-    The index-list rotation restarts at the first set in every graph."""
+    The index-list rotation restarts at the first set in every graph.  keep: the captured
+    graph stays inspectable (graph_kernel_nodes)."""
     import torch
     if idx_turn is not None:
         idx_turn[0] = 0
-    g = torch.cuda.CUDAGraph()
+    g = torch.cuda.CUDAGraph(keep_graph=keep)
     with torch.cuda.graph(g):
         for _ in range(n):
             fn()
+    if keep:
+        g.instantiate()
     return g
+
+
+def graph_kernel_nodes(g):
+    """Kernel launches recorded in a graph captured with keep=True.  The captured steps call
+    only this library, so every kernel node is one of its kernels."""
+    from cuda.bindings import runtime as rt
+    h = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+    err, _, n = rt.cudaGraphGetNodes(h, 0)
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaGraphGetNodes: {err}")
+    err, nodes, n = rt.cudaGraphGetNodes(h, n)
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaGraphGetNodes: {err}")
+    kernels = 0
+    for node in nodes[:n]:
+        err, kind = rt.cudaGraphNodeGetType(node)
+        if err != rt.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaGraphNodeGetType: {err}")
+        kernels += kind == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+    return kernels
 
 
 def _seq_len(name, args):
@@ -598,8 +620,11 @@ def measure_config(name, args, device, rank, world, clocks, peaks, peak_kind, sr
     # through); the loops replay K / G of them, so exactly K steps run.
     K = args.steps
     G = steps_per_graph(K, len(idx_sets))
-    g_chained = capture(chained_step, G, idx_turn)
-    g_fused = capture(fused_step, G, idx_turn)
+    g_chained = capture(chained_step, G, idx_turn, keep=True)
+    g_fused = capture(fused_step, G, idx_turn, keep=True)
+    # kernels per step, counted in the captured graphs (the index-list attend merges inside
+    # its clusters when they fit, so its step has no combine kernel)
+    per_step = {"chained": graph_kernel_nodes(g_chained) / G, "fused": graph_kernel_nodes(g_fused) / G}
     for _ in range(max(1, -(-args.warmup // G))):
         g_chained.replay()
         g_fused.replay()
@@ -635,7 +660,7 @@ def measure_config(name, args, device, rank, world, clocks, peaks, peak_kind, sr
     fused_ms, fused_value = aggregate(f_start.elapsed_time(f_stop) / K, acc["total"], device)
     # the step the line reports: whichever path (chained or fused) is faster on this workload
     best = "fused" if fused_ms < ms else "chained"
-    launches = K * (3 if best == "fused" else 4)
+    launches = int(round(K * per_step[best]))
 
     # Each stage alone, Kb times back to back in one graph (stage time = graph time / Kb),
     # and the attend call (attend + split-L combine) the same way: its duration as it runs
@@ -801,16 +826,20 @@ def measure_config(name, args, device, rank, world, clocks, peaks, peak_kind, sr
     c_ms, c_value = timed_cold(Kc)
     assert int(status.item()) == 0, m.status_string(int(status.item()))
 
-    roofline = attend_roofline(acc, att_ms, peaks, peak_kind, TRAFFIC.get((name, src_hash)))
+    in_cluster = per_step["chained"] < 4  # absorb, attend, up-projection: no combine kernel
+    roofline = attend_roofline(acc, att_ms, peaks, peak_kind, TRAFFIC.get((name, src_hash)),
+                               "attend_kernel, merging in its clusters (mla_attend_indexed)" if in_cluster
+                               else "attend_kernel + combine_kernel (mla_attend_*)")
     label = name if args.batch is None and args.seq_len is None else \
         f"{name} at a profiling size (B={B}, rows={args.seq_len})"
     rec = {
         "workload": arm_config(wl, label, world),
         "value": fused_value if best == "fused" else value, "unit": UNIT,
         "ms_per_step": fused_ms if best == "fused" else ms, "steps": K, "step_path": best,
-        "paths": {"chained": {"ms_per_step": ms, "value": value,
-                              "kernels": "absorb, attend, split-L combine, up-projection"},
-                  "fused": {"ms_per_step": fused_ms, "value": fused_value,
+        "paths": {"chained": {"ms_per_step": ms, "value": value, "kernels_per_step": per_step["chained"],
+                              "kernels": "absorb, attend, split-L merge (a combine kernel, or inside the "
+                                         "attend kernel's clusters for index lists), up-projection"},
+                  "fused": {"ms_per_step": fused_ms, "value": fused_value, "kernels_per_step": per_step["fused"],
                             "kernels": "absorb, attend, split-L merge fused with the up-projection",
                             "attend_and_merge_up_ms": attend_up_ms}},
         "stages_ms": {"absorb_q": stage[0], "attend": stage[1], "up_proj": stage[2], "attend_chained": att_ms},

@@ -119,6 +119,12 @@ mla_status mla_attend_paged(const uint16_t *q_tilde, const uint16_t *pool, const
  *                              producer below emits).
  *   seq_lens [B] int32 or NULL  as for mla_attend_dense (used to validate indices)
  * An out-of-range entry sets MLA_ERR_INDEX.  K >= 1.
+ * Each list is split over C = min(SMs / (B * Q), ceil(K / 64)) CTAs.  When C <= 8 and a
+ * cluster of C CTAs per list fits the device for every list at once (32 lists of 2,048
+ * entries on a B200: clusters of 4), the CTAs of a list run as one thread-block cluster
+ * and merge their partials inside the attend kernel: one kernel per call.  Otherwise a
+ * combine kernel follows, as for mla_attend_dense.  The workspace is used either way, and
+ * the results are the same bits.
  */
 mla_status mla_attend_indexed(const uint16_t *q_tilde, const uint16_t *cache, const int32_t *indices,
                               const int32_t *seq_lens, int B, int Q, int H, int R, int Lmax, int K,

@@ -84,7 +84,6 @@ int device_sm_count() {
   return sm_count_for(dev);
 }
 
-// Shared validation and launch for the three attend modes.
 // Shared validation and launch for the three attend modes.  With w_uv / out given, the
 // split-L merge runs fused with the up-projection (o_latent optional); without, the combine
 // writes o_latent (required).
@@ -158,9 +157,16 @@ static mla_status attend_common(int mode, const uint16_t *q_tilde, const uint16_
     const int nt = (K + 63) / 64;
     const int per_list = std::min(sms / lists, nt);
     p.groups = per_list >= 1 ? per_list * lists : sms;
+    // When a list's CTAs fit one thread-block cluster and all the clusters can be resident
+    // at once, they merge their partials in distributed shared memory (no partial stores,
+    // no combine kernel).  The fused up-projection path keeps the workspace partials.
+    p.cluster = 0;
+    if (!fused && per_list >= 1 && per_list <= 8 && attend_indexed_cluster_capacity(per_list) >= lists)
+      p.cluster = per_list;
   } else {
     p.group_size = Q;
     p.groups = std::max(1, sms / Q);
+    p.cluster = 0;
   }
   p.scale_log2 = scale * 1.4426950408889634f;
   const size_t slots = attend_slots(B, Q, sms);

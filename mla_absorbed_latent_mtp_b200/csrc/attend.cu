@@ -9,7 +9,8 @@
 // the same tiles at the same time, so all but the first read hit L2), or one CTA per
 // (sequence, query) list for the indexed mode.  Each segment leaves an unnormalised
 // partial (O, running max m, running sum l) in the workspace; the combine kernel merges
-// them with their log-sum-exp weights.
+// them with their log-sum-exp weights -- or, for index lists whose CTAs run as one
+// thread-block cluster per list, the cluster merges them itself after a cluster barrier.
 //
 // Per CTA (384 threads): warp 0 loads (one TMA copy per ring slot for dense/paged rows,
 // one for q~; 16-byte async copies for indexed rows, shared with warp 11), warp 1 issues
@@ -684,6 +685,161 @@ __device__ void softmax_role(const AttendParams &p, const Shared &sh, uint32_t t
   }
 }
 
+// ------------------------------------------------------------------ cluster merge (indexed)
+// The C CTAs of a cluster split one index list into C segments and write their partials to
+// the workspace as usual.  After one cluster barrier (release / acquire at cluster scope:
+// the partials are visible to the whole cluster) CTA `rank` merges heads
+// [rank * 64 / C, (rank + 1) * 64 / C) of the list from the C partials, which are still in
+// L2, and writes o_latent and lse: no combine kernel, and no wait on CTAs outside the
+// cluster (its CTAs are co-scheduled).  The merge is the combine kernel's, step for step --
+// partials in group order, in chunks of kMergeChunk, each chunk raising the running max M
+// and rescaling by 2^(M_old - M), then O / l and lse = (M + log2 l) ln 2 -- so the two
+// paths round identically.  Run by the eight softmax warps; every thread of the CTA takes
+// part in the cluster barrier (all reach it: every wait before it is bounded).
+constexpr int kMaxCluster = 8;
+constexpr int kMergeChunk = 3;
+constexpr int kMergeChunks = (kMaxCluster + kMergeChunk - 1) / kMergeChunk;
+constexpr int kCoef = 16;  // per head: kMergeChunks rescale factors, kMaxCluster weights, 1 / l
+static_assert(kMergeChunks + kMaxCluster + 1 <= kCoef, "merge coefficients");
+
+// Phase 1, one thread per head of this rank: the merge coefficients (all C partials' m and l
+// are loaded first, then folded chunk by chunk as the combine does).  Loads bypass L1: the
+// partials were written by other SMs during this kernel.
+template <int CC>
+__device__ __forceinline__ void merge_coefficients(const AttendParams &p, float *coef, int v, int h, int t) {
+  float mk[kMergeChunks * kMergeChunk], lk[kMergeChunks * kMergeChunk];
+#pragma unroll
+  for (int k = 0; k < kMergeChunks * kMergeChunk; ++k) {
+    mk[k] = -INFINITY;
+    lk[k] = 0.f;
+  }
+#pragma unroll
+  for (int k = 0; k < CC; ++k) {
+    const long long row = split::partial_slot(p, kModeIndexed, (long long)v * CC + k, v, 0) * kRows + h;
+    mk[k] = __ldcg(p.part_m + row);
+    lk[k] = __ldcg(p.part_l + row);
+  }
+  float *cf = coef + t * kCoef;
+  float M = -INFINITY, den = 0.f;
+#pragma unroll
+  for (int c = 0; c < kMergeChunks; ++c) {
+    if (c * kMergeChunk >= CC) break;
+    float mx = M;
+#pragma unroll
+    for (int j = 0; j < kMergeChunk; ++j) mx = fmaxf(mx, mk[c * kMergeChunk + j]);
+    if (mx == -INFINITY) {
+      cf[c] = -1.f;
+      continue;
+    }
+    const float a = exp2f(M - mx);  // 0 when M was -inf
+    cf[c] = a;
+    den *= a;
+#pragma unroll
+    for (int j = 0; j < kMergeChunk; ++j) {
+      const int k = c * kMergeChunk + j;
+      const float w = exp2f(mk[k] - mx);  // 0 for empty partials (m = -inf)
+      if (k < kMaxCluster) cf[kMergeChunks + k] = w;
+      if (w == 0.f) continue;
+      den += w * lk[k];
+    }
+    M = mx;
+  }
+  const bool good = (M != -INFINITY) && den > 0.f;
+  cf[kMergeChunks + kMaxCluster] = good ? 1.f / den : 0.f;
+  if (p.lse != nullptr)
+    p.lse[(long long)v * kRows + h] = good ? (M + log2f(den)) * 0.69314718055994530942f : -INFINITY;
+}
+
+// Phase 2, 256 threads over this rank's (head, 4 latents) elements: the loads of U elements
+// (U * CC float4, 16 or fewer) are issued together before any is used, then each element is
+// folded with the coefficients exactly as the combine folds its partials.
+template <int CC>
+__device__ __forceinline__ void merge_rows(const AttendParams &p, const float *coef, int v, int h0, int nh, int t) {
+  constexpr int U = (16 / CC) > 8 ? 8 : (16 / CC);
+  constexpr int kStride = 32 * kSoftmaxWarps;
+  const float *part[CC];
+#pragma unroll
+  for (int k = 0; k < CC; ++k)
+    part[k] = p.part_o + split::partial_slot(p, kModeIndexed, (long long)v * CC + k, v, 0) * kRows * kLatent;
+  const int total = nh * (kLatent / 4);  // a multiple of 128: every warp's elements are all in or all out
+  for (int e0 = t; e0 < total; e0 += U * kStride) {
+    float4 o[U][CC];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int e = e0 + u * kStride;
+      if (e < total) {
+        const int off = (h0 + e / (kLatent / 4)) * kLatent + (e % (kLatent / 4)) * 4;
+#pragma unroll
+        for (int k = 0; k < CC; ++k) o[u][k] = __ldcg(reinterpret_cast<const float4 *>(part[k] + off));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int e = e0 + u * kStride;
+      if (e >= total) continue;
+      const int hl = e / (kLatent / 4), lat = (e % (kLatent / 4)) * 4;
+      const float *cf = coef + hl * kCoef;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < kMergeChunks; ++c) {
+        if (c * kMergeChunk >= CC) break;
+        const float a = cf[c];
+        if (a < 0.f) continue;  // every partial of the chunk is empty
+        acc.x *= a;
+        acc.y *= a;
+        acc.z *= a;
+        acc.w *= a;
+#pragma unroll
+        for (int j = 0; j < kMergeChunk; ++j) {
+          const int k = c * kMergeChunk + j;
+          if (k >= CC) break;
+          const float w = cf[kMergeChunks + k];
+          if (w == 0.f) continue;  // an empty partial's O is never used
+          acc.x += w * o[u][k].x;
+          acc.y += w * o[u][k].y;
+          acc.z += w * o[u][k].z;
+          acc.w += w * o[u][k].w;
+        }
+      }
+      const float inv = cf[kMergeChunks + kMaxCluster];
+      uint2 outv;
+      outv.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+      outv.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2 *>(p.o_latent + ((long long)v * kRows + h0 + hl) * kLatent + lat) = outv;
+    }
+  }
+}
+
+template <int CC>
+__device__ void cluster_merge_n(const AttendParams &p, const Shared &sh, int t) {
+  const int rank = (int)cluster_ctarank();
+  const int v = blockIdx.x / CC;  // the list: b * Q + i
+  const int h0 = rank * kHeads / CC, nh = (rank + 1) * kHeads / CC - h0;
+  // per-head coefficients, staged over the q~ area (free by now): for chunk c the rescale
+  // factor a_c (-1: the chunk is skipped, all its partials empty), the weights w_k, 1 / l
+  float *coef = reinterpret_cast<float *>(sh.base + kOffQt);
+  if (t < nh) merge_coefficients<CC>(p, coef, v, h0 + t, t);
+  named_bar_sync(3, 32 * kSoftmaxWarps);
+  merge_rows<CC>(p, coef, v, h0, nh, t);
+}
+
+__device__ void cluster_merge(const AttendParams &p, const Shared &sh, int warp, int lane) {
+  cluster_sync_all();  // every partial of the cluster's list is in the workspace
+  if (warp >= 2 && warp < 2 + kSoftmaxWarps && !*sh.abort_flag) {
+    const int t = (warp - 2) * 32 + lane;  // 0..255
+    switch (p.cluster) {
+      case 1: cluster_merge_n<1>(p, sh, t); break;
+      case 2: cluster_merge_n<2>(p, sh, t); break;
+      case 3: cluster_merge_n<3>(p, sh, t); break;
+      case 4: cluster_merge_n<4>(p, sh, t); break;
+      case 5: cluster_merge_n<5>(p, sh, t); break;
+      case 6: cluster_merge_n<6>(p, sh, t); break;
+      case 7: cluster_merge_n<7>(p, sh, t); break;
+      default: cluster_merge_n<8>(p, sh, t); break;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ kernel
 template <int kMode>
 // Bounds for 384 threads: eleven warps put three on some SM sub-partitions, whose 16K
@@ -795,6 +951,9 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  if constexpr (kMode == kModeIndexed) {
+    if (p.cluster > 0) cluster_merge(p, sh, warp, lane);
+  }
 }
 
 // ------------------------------------------------------------------ combine
@@ -808,6 +967,7 @@ __global__ void __launch_bounds__(384, 1)
 // table the attend kernel wrote.
 constexpr int kCombineHeads = 2;
 constexpr int kCombineChunk = 3;
+static_assert(kCombineChunk == kMergeChunk, "the cluster merge rounds like the combine");
 
 __global__ void __launch_bounds__(128, 8) combine_kernel(const AttendParams p, int mode) {
   grid_dep_launch();
@@ -979,11 +1139,64 @@ static cudaError_t launch_attend_mode(const CUtensorMap &tm_cache, const CUtenso
     configured_device = dev;
   }
   const int grid = p.groups * p.group_size;
+  if (kMode == kModeIndexed && p.cluster > 0) {
+    // one cluster per index list; the cluster merges its partials and writes o_latent / lse
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(attend::kThreads);
+    cfg.dynamicSmemBytes = attend::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)p.cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, attend::attend_kernel<kMode>, tm_cache, tm_qt, p);
+  }
   cudaError_t e = launch_chained(attend::attend_kernel<kMode>, dim3(grid), dim3(attend::kThreads), attend::kSmemBytes,
                                  stream, tm_cache, tm_qt, p);
   if (e != cudaSuccess || !with_combine) return e;
   dim3 cgrid(p.B * p.Q, kHeads / attend::kCombineHeads);
   return launch_chained(attend::combine_kernel, cgrid, dim3(128), 0, stream, p, (int)kMode);
+}
+
+int attend_indexed_cluster_capacity(int csize) {
+  if (csize < 1 || csize > attend::kMaxCluster) return 0;
+  static int cached_device = -1;
+  static int cached[attend::kMaxCluster + 1];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cached_device != dev) {
+    for (int c = 0; c <= attend::kMaxCluster; ++c) cached[c] = -1;
+    if (cudaFuncSetAttribute(attend::attend_kernel<kModeIndexed>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             attend::kSmemBytes) != cudaSuccess)
+      return 0;
+    cached_device = dev;
+  }
+  if (cached[csize] < 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(csize);
+    cfg.blockDim = dim3(attend::kThreads);
+    cfg.dynamicSmemBytes = attend::kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, attend::attend_kernel<kModeIndexed>, &cfg) != cudaSuccess) {
+      cudaGetLastError();  // not an error of the caller's stream: no cluster launch
+      n = 0;
+    }
+    cached[csize] = n;
+  }
+  return cached[csize];
 }
 
 cudaError_t launch_attend(int mode, const CUtensorMap &tm_cache, const CUtensorMap &tm_qt, const AttendParams &p,

@@ -28,6 +28,9 @@ struct AttendParams {
   int B, Q, Lmax, max_pages, num_pages, K;
   int groups;                 // G: CTA groups that split the tile list
   int group_size;             // CTAs per group: Q (dense/paged, one per query) or 1 (indexed)
+  int cluster;                // indexed: CTAs per list, launched as one thread-block cluster that
+                              // merges its partials in distributed shared memory and writes
+                              // o_latent / lse itself (no combine); 0: partials to the workspace
   float scale_log2;           // softmax scale * log2(e)
   float *part_o;              // [slots, H, R] unnormalised partial outputs
   float *part_m;              // [slots, H] running max (log2 units)
@@ -43,9 +46,13 @@ struct AttendParams {
 size_t attend_slots(int B, int Q, int sms);
 size_t attend_workspace_bytes_for(int B, int Q, int sms);
 
-// The attend kernel, then (with_combine) the split-L combine that writes o_latent / lse.
+// The attend kernel, then (with_combine, and p.cluster == 0) the split-L combine that
+// writes o_latent / lse.
 cudaError_t launch_attend(int mode, const CUtensorMap &tm_cache, const CUtensorMap &tm_qt,
                           const AttendParams &p, cudaStream_t stream, bool with_combine = true);
+// Clusters of `csize` indexed-mode attend CTAs (one CTA per SM) that can be resident at once
+// on the current device (0 when the launch configuration is not possible).
+int attend_indexed_cluster_capacity(int csize);
 // The split-L merge fused with the W_UV up-projection: out [B*Q, H, D] from the attend
 // kernel's partials (o_latent / lse in p written too when non-null).
 cudaError_t launch_merge_up(const CUtensorMap &tm_w, const AttendParams &p, int mode, uint16_t *out,
