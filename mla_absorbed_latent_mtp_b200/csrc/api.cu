@@ -48,14 +48,14 @@ bool make_map(CUtensorMap *map, const void *ptr, int rank, const uint64_t *dims,
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int sm_count_for(int dev) {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];  // 0: not read yet (concurrent first calls both read it)
   if (dev < 0 || dev >= 64) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 // W_UV[h][d][r] for the fused merge + up-projection: dims {R, D, H}, boxes of 64 r x 128 d.

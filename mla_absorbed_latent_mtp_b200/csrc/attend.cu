@@ -27,6 +27,9 @@
 #include <math.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "internal.h"
 #include "sm100.cuh"
@@ -1129,15 +1132,9 @@ size_t attend_workspace_bytes_for(int B, int Q, int sms) {
 template <int kMode>
 static cudaError_t launch_attend_mode(const CUtensorMap &tm_cache, const CUtensorMap &tm_qt, const AttendParams &p,
                                       cudaStream_t stream, bool with_combine) {
-  static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(attend::attend_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         attend::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  static std::atomic<int> configured_device{-1};
+  const cudaError_t e0 = set_smem_limit_once(attend::attend_kernel<kMode>, attend::kSmemBytes, configured_device);
+  if (e0 != cudaSuccess) return e0;
   const int grid = p.groups * p.group_size;
   if (kMode == kModeIndexed && p.cluster > 0) {
     // one cluster per index list; the cluster merges its partials and writes o_latent / lse
@@ -1166,18 +1163,17 @@ static cudaError_t launch_attend_mode(const CUtensorMap &tm_cache, const CUtenso
 
 int attend_indexed_cluster_capacity(int csize) {
   if (csize < 1 || csize > attend::kMaxCluster) return 0;
-  static int cached_device = -1;
-  static int cached[attend::kMaxCluster + 1];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cached_device != dev) {
-    for (int c = 0; c <= attend::kMaxCluster; ++c) cached[c] = -1;
-    if (cudaFuncSetAttribute(attend::attend_kernel<kModeIndexed>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             attend::kSmemBytes) != cudaSuccess)
-      return 0;
-    cached_device = dev;
-  }
-  if (cached[csize] < 0) {
+  // per (device, cluster size), computed once; the lock makes concurrent first calls safe
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto it = cache.find({dev, csize});
+  if (it != cache.end()) return it->second;
+  int n = 0;
+  if (cudaFuncSetAttribute(attend::attend_kernel<kModeIndexed>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           attend::kSmemBytes) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(csize);
     cfg.blockDim = dim3(attend::kThreads);
@@ -1189,14 +1185,11 @@ int attend_indexed_cluster_capacity(int csize) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, attend::attend_kernel<kModeIndexed>, &cfg) != cudaSuccess) {
-      cudaGetLastError();  // not an error of the caller's stream: no cluster launch
-      n = 0;
-    }
-    cached[csize] = n;
+    if (cudaOccupancyMaxActiveClusters(&n, attend::attend_kernel<kModeIndexed>, &cfg) != cudaSuccess) n = 0;
   }
-  return cached[csize];
+  cudaGetLastError();  // a failed query is not an error of the caller's: the combine path runs
+  cache[{dev, csize}] = n;
+  return n;
 }
 
 cudaError_t launch_attend(int mode, const CUtensorMap &tm_cache, const CUtensorMap &tm_qt, const AttendParams &p,

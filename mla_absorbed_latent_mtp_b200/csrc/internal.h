@@ -6,6 +6,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 namespace mla {
@@ -97,6 +98,18 @@ cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current device, once per
+// device switch (`configured` remembers the device it was last set on).  Safe from several
+// host threads: the attribute call is idempotent, so concurrent first calls may both make it.
+template <typename... KArgs>
+cudaError_t set_smem_limit_once(void (*kernel)(KArgs...), int bytes, std::atomic<int> &configured) {
+  int dev = 0;
+  if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return e;
+  if (configured.load(std::memory_order_acquire) == dev) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) configured.store(dev, std::memory_order_release);
+  return e;
 }
 // Records e as the calling thread's last CUDA error; returns MLA_ERR_CUDA (MLA_OK for success).
 int32_t record_cuda_error(cudaError_t e);

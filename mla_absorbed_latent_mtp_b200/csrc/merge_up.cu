@@ -350,15 +350,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_merge_up(const CUtensorMap &tm_w, const AttendParams &p, int mode, uint16_t *out,
                             cudaStream_t stream) {
-  static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(mergeup::merge_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         mergeup::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  static std::atomic<int> configured_device{-1};
+  const cudaError_t e0 = set_smem_limit_once(mergeup::merge_up_kernel, mergeup::kSmemBytes, configured_device);
+  if (e0 != cudaSuccess) return e0;
   const int n = p.B * p.Q;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(mergeup::kChunks, kHeads, (n + mergeup::kNTile - 1) / mergeup::kNTile);

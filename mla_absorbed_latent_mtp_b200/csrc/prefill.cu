@@ -327,15 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_prefill(const CUtensorMap &tm_k, const CUtensorMap &tm_v, const uint16_t *q, uint16_t *out,
                            float *lse, int B, int L, float scale, int32_t *status, cudaStream_t stream) {
-  static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(prefill::prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         prefill::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  static std::atomic<int> configured_device{-1};
+  const cudaError_t e0 = set_smem_limit_once(prefill::prefill_kernel, prefill::kSmemBytes, configured_device);
+  if (e0 != cudaSuccess) return e0;
   prefill::Params p{q, out, lse, B, L, scale * 1.4426950408889634f, status};
   const int nqb = (L + prefill::kQBlock - 1) / prefill::kQBlock;
   return launch_chained(prefill::prefill_kernel, dim3(nqb, kHeads, B), dim3(prefill::kThreads), prefill::kSmemBytes,

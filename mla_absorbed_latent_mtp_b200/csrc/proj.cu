@@ -169,15 +169,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <bool kAMajorMN>
 static cudaError_t launch_proj_t(const CUtensorMap &tm_w, const CUtensorMap &tm_x, const proj::Params &p,
                                  cudaStream_t stream) {
-  static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(proj::proj_kernel<kAMajorMN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         proj::kSmemLimit);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  static std::atomic<int> configured_device{-1};
+  const cudaError_t e0 = set_smem_limit_once(proj::proj_kernel<kAMajorMN>, proj::kSmemLimit, configured_device);
+  if (e0 != cudaSuccess) return e0;
   dim3 grid(p.H, p.M_total / proj::kBM, (p.n + p.n_tile - 1) / p.n_tile);
   return launch_chained(proj::proj_kernel<kAMajorMN>, grid, dim3(proj::kThreads), proj::smem_bytes(p.stages, p.n_tile),
                         stream, tm_w, tm_x, p);
