@@ -43,11 +43,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of one attend launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
 # ncu capture summarised in profiles/, keyed by the hash of the kernel source it was taken on.
 TRAFFIC = {
-    ("tiny_dense_decode", "3a31264b08832ba4"): 398_080,
-    ("dense_decode", "3a31264b08832ba4"): 277_780_480,
-    ("mtp_verify", "3a31264b08832ba4"): 556_406_016,
-    ("ragged_paged_decode", "3a31264b08832ba4"): 4_378_480_640,
-    ("indexed_sparse_decode", "3a31264b08832ba4"): 71_251_456,
+    ("tiny_dense_decode", "9b3bd05e2802578a"): 398_080,
+    ("dense_decode", "9b3bd05e2802578a"): 277_927_936,
+    ("mtp_verify", "9b3bd05e2802578a"): 556_837_376,
+    ("ragged_paged_decode", "9b3bd05e2802578a"): 4_382_152_448,
+    ("indexed_sparse_decode", "9b3bd05e2802578a"): 71_590_656,
 }
 
 
