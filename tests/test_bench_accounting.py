@@ -100,3 +100,65 @@ def test_graph_batches_time_exactly_k_steps(K, n_rot):
     assert 1 <= G <= 32 and K % G == 0
     if any(K % g == 0 and g % n_rot == 0 for g in range(1, min(K, 32) + 1)):
         assert G % n_rot == 0
+
+
+class _FakeRuntime:
+    """Stands in for the CUDA runtime binding: a graph of the given node kinds."""
+
+    class cudaError_t:
+        cudaSuccess = 0
+        cudaErrorInvalidValue = 1
+
+    class cudaGraphNodeType:
+        cudaGraphNodeTypeKernel = "kernel"
+        cudaGraphNodeTypeMemcpy = "memcpy"
+        cudaGraphNodeTypeEventRecord = "event"
+
+    def __init__(self, kinds, fail=False):
+        self.kinds, self.fail, self.handles = kinds, fail, []
+
+    def cudaGraph_t(self, init_value):
+        self.handles.append(init_value)
+        return ("graph", init_value)
+
+    def cudaGraphGetNodes(self, h, n):
+        assert h == ("graph", 1234)
+        if self.fail:
+            return self.cudaError_t.cudaErrorInvalidValue, [], 0
+        # a count query first (n = 0), then the nodes themselves
+        return self.cudaError_t.cudaSuccess, list(range(len(self.kinds)))[:n], len(self.kinds)
+
+    def cudaGraphNodeGetType(self, node):
+        return self.cudaError_t.cudaSuccess, self.kinds[node]
+
+
+class _FakeGraph:
+    def raw_cuda_graph(self):
+        return 1234
+
+
+def _with_runtime(monkeypatch, rt):
+    import sys
+    import types
+    pkg = types.ModuleType("cuda.bindings")
+    pkg.runtime = rt
+    monkeypatch.setitem(sys.modules, "cuda.bindings", pkg)
+    monkeypatch.setitem(sys.modules, "cuda.bindings.runtime", rt)
+
+
+def test_launch_count_counts_kernel_nodes_only(monkeypatch):
+    """gpu_launches comes from the captured step graph: kernel nodes counted, copies and
+    event nodes not."""
+    K = _FakeRuntime.cudaGraphNodeType
+    kinds = [K.cudaGraphNodeTypeKernel] * 3 + [K.cudaGraphNodeTypeMemcpy, K.cudaGraphNodeTypeEventRecord] + \
+        [K.cudaGraphNodeTypeKernel] * 4
+    rt = _FakeRuntime(kinds)
+    _with_runtime(monkeypatch, rt)
+    assert bench.graph_kernel_nodes(_FakeGraph()) == 7
+    assert rt.handles == [1234]
+
+
+def test_launch_count_fails_loudly(monkeypatch):
+    _with_runtime(monkeypatch, _FakeRuntime([], fail=True))
+    with pytest.raises(RuntimeError):
+        bench.graph_kernel_nodes(_FakeGraph())
